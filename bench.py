@@ -1,0 +1,420 @@
+#!/usr/bin/env python3
+"""Benchmark of Re-ttention's reshaped block-sparse attention hot path on B200.
+
+One step = one pass of the whole hot path over one calibration cycle of the
+workload: build the CSR block index of the static mask, one calibration
+(full-attention) step on X_0, then the workload's sparse steps on the drifted
+inputs X_1..X_n with step distance k = 1..n.  Inputs (all steps' Q/K/V) are
+resident in HBM when the timed region starts; each step's inputs (>= 205 MB
+for the default workload) exceed the 126 MB L2, so no explicit flush is done.
+
+Metric: executed-block TFLOP/s (4 * block^2 * d * kept blocks * B * H per
+attention call, true d; calibration executes every block).  The line also
+carries per-kernel latency/TFLOP/s, the roofline object of the dominant
+kernel, the CPU oracle baseline, the end-to-end number through the public API
+with host buffers, and the SM clocks seen during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+Multi-GPU (weak scaling, independent replicas, no data-path collective):
+    python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_diffusion_rt_b200 import inputs  # noqa: E402
+
+METRIC = "sparse-step attention latency & TFLOP/s (executed blocks), % bf16 peak, 1 B200"
+DEFAULT_WORKLOAD = "cogvideox"
+KERNEL_SOURCES = ("attn_kernel.cuh", "ptx.cuh")
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_attention_diffusion_rt_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (its 'source_hash' line matches), else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", txt)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def executed_flops(w: inputs.Workload, nnz_per_head: int) -> float:
+    return 4.0 * w.block * w.block * w.d * nnz_per_head * w.B * w.H
+
+
+# ---------------------------------------------------------------------------
+# the step
+# ---------------------------------------------------------------------------
+
+class Step:
+    """One calibration cycle through the C ABI, with per-kernel CUDA events."""
+
+    def __init__(self, w, mask_dev, qkv_steps, rt):
+        self.w, self.mask, self.qkv, self.rt = w, mask_dev, qkv_steps, rt
+        q = qkv_steps[0][0]
+        self.o = [torch.empty_like(q) for _ in qkv_steps]
+        self.rho = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=q.device)
+        self.r = torch.empty_like(q)
+        n = len(qkv_steps)
+        self.ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        self.times = {"calibrate": [], "sparse": []}
+        self.launches = 0
+
+    def run(self, record=False):
+        rt, w = self.rt, self.w
+        idx = rt.rt_build_block_index(self.mask)
+        self.launches += 3
+        q, k, v = self.qkv[0]
+        if record:
+            self.ev[0][0].record()
+        rt.rt_calibrate(q, k, v, idx, block=w.block, o=self.o[0], rho=self.rho, r=self.r)
+        if record:
+            self.ev[0][1].record()
+        self.launches += 1
+        for s in range(1, len(self.qkv)):
+            q, k, v = self.qkv[s]
+            if record:
+                self.ev[s][0].record()
+            rt.rt_sparse_step(q, k, v, idx, self.rho, self.r, block=w.block, lam=w.lam, step_distance=s,
+                              o=self.o[s])
+            if record:
+                self.ev[s][1].record()
+            self.launches += 1
+        self.idx = idx
+
+    def collect(self):
+        self.times["calibrate"].append(self.ev[0][0].elapsed_time(self.ev[0][1]))
+        for s in range(1, len(self.qkv)):
+            self.times["sparse"].append(self.ev[s][0].elapsed_time(self.ev[s][1]))
+
+
+def cpu_oracle_sample(w, qkv_steps_cpu, mask, budget_s=15.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload:
+    query blocks of head (0, 0), sparse step first, then calibration rows, until
+    ~budget_s of CPU time.  Returns (executed-block TFLOP/s, description, cores)."""
+    from oracle import reference as ref
+    q0, k0, v0 = (x[0, 0].double().numpy() for x in qkv_steps_cpu[0])
+    q1, k1, v1 = (x[0, 0].double().numpy() for x in qkv_steps_cpu[min(1, len(qkv_steps_cpu) - 1)])
+    L, blk = w.L, w.block
+    nqb = w.nqb
+    bm = mask[0]
+    flops, n_sp, n_cal = 0.0, 0, 0
+    t0 = time.perf_counter()
+    order = np.random.default_rng(0).permutation(nqb)
+    for qb in order:
+        rows = np.arange(qb * blk, min(L, (qb + 1) * blk))
+        O, RHO, R = ref.calibrate_rows_ref(q0, k0, v0, bm, blk, rows)
+        flops += 4.0 * blk * blk * w.d * w.nkb
+        n_cal += 1
+        ref.sparse_step_rows_ref(q1, k1, v1, bm, blk, rows, RHO, R, w.lam, 1)
+        flops += 4.0 * blk * blk * w.d * int(bm[qb].sum())
+        n_sp += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"head (0,0) of {w.name}: {n_cal} query blocks calibrated + sparse-stepped "
+            f"({n_cal}/{w.B * w.H * nqb} of the cycle's calibration units) in {dt:.1f} s; "
+            f"executed-block FLOPs of the sample / CPU time")
+    return flops / dt / 1e12, desc, cores
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[args.workload]
+    steps = inputs.qkv_steps(w, 2, device="cpu")
+    mask = inputs.block_mask(w)
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, desc, cores = cpu_oracle_sample(w, steps, mask, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(v)
+    value = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block,
+                   "kept_blocks_per_row": w.kept, "sparse_steps": w.n_sparse_steps},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    from sparse_attention_diffusion_rt_b200 import rt
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    rt.load_library()
+    w = inputs.WORKLOADS[args.workload]
+    peaks = load_peaks()
+    n_steps = 1 + w.n_sparse_steps
+    qkv = inputs.qkv_steps(w, n_steps, device=dev)
+    mask_np = inputs.block_mask(w)
+    mask = torch.from_numpy(mask_np).to(dev)
+    nnz = int(mask_np.sum())
+    cal_flops = executed_flops(w, w.nqb * w.nkb)
+    sp_flops = executed_flops(w, nnz)
+    step_flops = cal_flops + w.n_sparse_steps * sp_flops
+    step = Step(w, mask, qkv, rt)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    st = rt.rt_check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {rt.rt_status_string(st)}")
+
+    # ---- device-timed region: all K steps, events on the launching stream
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    step.launches = 0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(args.steps):
+        step.run()
+    end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    launches = step.launches
+    st = rt.rt_check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in timed region: {rt.rt_status_string(st)}")
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- per-kernel timing: separate pass, each kernel bracketed by events
+    step.times = {"calibrate": [], "sparse": []}
+    for _ in range(max(3, min(args.steps, 10))):
+        step.run(record=True)
+        torch.cuda.synchronize()
+        step.collect()
+    cal_ms = float(np.median(step.times["calibrate"]))
+    sp_ms = float(np.median(step.times["sparse"]))
+    cal_tf = cal_flops / (cal_ms * 1e-3) / 1e12
+    sp_tf = sp_flops / (sp_ms * 1e-3) / 1e12
+    share_cal = cal_ms / (cal_ms + w.n_sparse_steps * sp_ms)
+    dominant = ("calibrate", cal_ms, cal_flops, cal_tf) if share_cal >= 0.5 else ("sparse_step", sp_ms, sp_flops, sp_tf)
+    peak = peaks["bf16_tflops"]
+
+    def roof(tag, ms, fl, tf):
+        return {"kernel": tag, "bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                "frac": tf / peak, "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+                "peak_source": peaks["source"] + " (burst)", "algorithmic_flops_per_launch": fl,
+                "launch_ms": ms, "traffic": profiled_traffic(tag, w.name)}
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = [tuple(x.cpu().pin_memory() for x in s) for s in qkv]
+        host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in step.o]
+        h2d = sum(x.numel() * x.element_size() for s in host_in for x in s)
+        d2h = sum(o.numel() * o.element_size() for o in host_out)
+        dev_in = [tuple(torch.empty_like(x) for x in s) for s in qkv]
+        step_e2e = Step(w, mask, dev_in, rt)
+        n_e2e = max(2, min(args.steps, 5))
+
+        def e2e_once():
+            for s_h, s_d in zip(host_in, dev_in):
+                for xh, xd in zip(s_h, s_d):
+                    xd.copy_(xh, non_blocking=True)
+            step_e2e.run()
+            for oh, od in zip(host_out, step_e2e.o):
+                oh.copy_(od, non_blocking=True)
+        e2e_once()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_once()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del host_in, host_out, dev_in, step_e2e
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        steps_cpu = [tuple(x.cpu() for x in qkv[0]), tuple(x.cpu() for x in qkv[1])]
+        v, desc, cores = cpu_oracle_sample(w, steps_cpu, mask_np, budget_s=args.cpu_budget)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block,
+                       "kept_blocks_per_row": w.kept, "sparsity": 1 - nnz / (w.nqb * w.nkb),
+                       "sparse_steps": w.n_sparse_steps, "lambda": w.lam,
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+            "step": "block index + 1 calibration + %d sparse steps" % w.n_sparse_steps,
+            "sparse_step": {"latency_us": sp_ms * 1e3, "tflops": sp_tf, "frac_of_peak": sp_tf / peak,
+                            "executed_gflop": sp_flops / 1e9},
+            "calibrate": {"latency_us": cal_ms * 1e3, "tflops": cal_tf, "frac_of_peak": cal_tf / peak,
+                          "executed_gflop": cal_flops / 1e9},
+            "roofline": roof(*dominant),
+            "roofline_sparse_step": roof("sparse_step", sp_ms, sp_flops, sp_tf),
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * rt.h -- C ABI of the B200 (sm_100a) implementation of Re-ttention's
+ * statistically reshaped static block-sparse attention.
+ *
+ * Source of the operations: "Re-ttention: Ultra Sparse Visual Generation via
+ * Attention Statistical Reshape" -- the summary page ("Approach") and the
+ * OpenReview discussion (replies to W1 of the three reviewers: the worked
+ * 4-key example, rho as the ratio of sparse to full softmax denominator, the
+ * residual of the masked tokens; reply to Q2: rho per head and per token;
+ * reply to Q4: the residual has the attention output's shape; reply to W2:
+ * static masks; reply to Pwod's W1: the ramp-up lambda).
+ *
+ * Notation, per batch b and head h, query row i, key j:
+ *   s_ij = c <q_i, k_j>, c = softmax_scale (0 selects 1/sqrt(d), true d)
+ *   M(i) = keys in the key blocks kept for i's query block; V(i) = keys j < L.
+ *
+ * Common conventions
+ *   - Every buffer is caller-owned device memory, except where a name starts
+ *     with h_ (host).  The library allocates nothing but one device status
+ *     word per device (a static __device__ variable).
+ *   - Q, K, V, O and R share one layout: element (b, h, l, t) is at
+ *     b*stride_b + h*stride_h + l*stride_l + t (elements; t contiguous).
+ *     Q, K, V and O are bf16; R is bf16 or fp32 (rt_attn_desc.r_dtype).
+ *     rho is fp32 [B, H, L] contiguous.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) unless stated otherwise.  They are stateless and
+ *     reentrant.  There is no CPU fallback.
+ *   - Host-side validation failures return a status and launch nothing.
+ *     Faults found on the device (a bad block index, a wait that ran past its
+ *     limit) never trap: the kernel records the first status in the device
+ *     status word, skips the affected work and returns; read it with
+ *     rt_check_device_error.
+ *   - Supported: 16 <= d <= 128 with d % 8 == 0 (d is padded to 64, 80, 96 or
+ *     128 inside the kernels), block in {64, 128}, strides multiples of 8
+ *     elements, pointers 16-byte aligned, 1 <= L and ceil(L/block) <= 4096.
+ *     Other shapes return RT_ERR_UNSUPPORTED.
+ */
+#ifndef RT_B200_H
+#define RT_B200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RT_API __attribute__((visibility("default")))
+#else
+#define RT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rt_status {
+  RT_OK = 0,
+  RT_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, negative size, inconsistent index */
+  RT_ERR_UNSUPPORTED = 2,      /* valid but outside the supported shapes above */
+  RT_ERR_CAPACITY = 3,         /* output array too small (rt_build_block_index) */
+  RT_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed; see rt_last_cuda_error */
+  RT_ERR_TIMEOUT = 5,          /* device: an mbarrier wait ran past its limit */
+  RT_ERR_BAD_INDEX = 6         /* device: row_ptr/col_idx out of range or not ascending */
+} rt_status;
+
+/* Ramp-up of the cached rho with the step distance k since calibration
+ * (reply to Pwod's W1: rho grows over denoising, lambda = 0.04 best).  The
+ * pages give no formula; all three equal rho at lambda = 0 or k = 0 and clamp
+ * at 1.  MUL_LINEAR is the default reading. */
+typedef enum rt_ramp {
+  RT_RAMP_MUL_LINEAR = 0, /* min(1, rho * (1 + lambda k)) */
+  RT_RAMP_ADD_LINEAR = 1, /* min(1, rho + lambda k)       */
+  RT_RAMP_GEOMETRIC = 2   /* min(1, rho * (1 + lambda)^k) */
+} rt_ramp;
+
+typedef enum rt_dtype { RT_BF16 = 0, RT_F32 = 1 } rt_dtype;
+
+typedef struct rt_attn_desc {
+  int32_t B, H, L, d;   /* batch, heads, tokens, head dimension */
+  int32_t block;        /* query and key block size: 64 or 128 */
+  int64_t stride_b, stride_h, stride_l; /* element strides shared by Q, K, V, O, R */
+  float softmax_scale;  /* c; 0 selects 1/sqrt(d) */
+  rt_dtype r_dtype;     /* residual R element type */
+} rt_attn_desc;
+
+/* CSR block index of the static mask (device arrays).  Rows are (hm, qb)
+ * flattened hm-major, hm in [0, Hm); Hm == 1 shares one mask across all
+ * batches and heads, Hm == H gives each head its own.  Row r lists its kept
+ * key blocks col_idx[row_ptr[r] .. row_ptr[r+1]) in strictly ascending order;
+ * row_ptr[0] == 0 and row_ptr[Hm*nqb] == nnz. */
+typedef struct rt_block_index {
+  int32_t Hm, nqb, nkb;   /* nqb == nkb == ceil(L / block) */
+  int64_t nnz;
+  const int32_t* row_ptr; /* device, Hm*nqb + 1 entries */
+  const int32_t* col_idx; /* device, nnz entries (may be NULL when nnz == 0) */
+} rt_block_index;
+
+/* Dense block mask -> CSR block index (the static mask is free at inference,
+ * reply to W2; the index is built once per mask).
+ *   d_mask      device u8 [Hm, nqb, nkb], nonzero = key block kept.
+ *   d_row_ptr   device i32 [Hm*nqb + 1], written: exclusive prefix sum of row counts.
+ *   d_col_idx   device i32 [col_capacity], written: kept key blocks, ascending per row.
+ *   h_nnz       host, receives the total number of kept blocks.
+ * Synchronises `stream` once to read nnz.  Returns RT_ERR_CAPACITY (and
+ * writes only the rows that fit) when nnz > col_capacity. */
+RT_API rt_status rt_build_block_index(const uint8_t* d_mask, int32_t Hm, int32_t nqb, int32_t nkb,
+                               int32_t* d_row_ptr, int32_t* d_col_idx, int64_t col_capacity,
+                               int64_t* h_nnz, void* stream);
+
+/* Calibration (full-attention) step.  For every (b, h, i):
+ *   O_i   = sum_{j in V(i)} e^{s_ij - m_i} v_j / Z_full          (bf16 out)
+ *   rho_i = Z_sp / Z_full                                        (fp32 out)
+ *   R_i   = sum_{j in V(i) \ M(i)} e^{s_ij - m_i} v_j / Z_full   (r_dtype out)
+ * with Z_full = sum_{V(i)} e^{s_ij - m_i}, Z_sp = sum_{M(i)} e^{s_ij - m_i},
+ * one shared row max m_i.  One tensor-core pass over all key blocks; the
+ * in-mask and out-of-mask sums and outputs are kept apart. */
+RT_API rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                       const rt_block_index* idx, void* o, float* rho, void* r, void* stream);
+
+/* Reshaped sparse step at step distance k >= 0 since the calibration:
+ *   O'_i = ramp(rho_i, lambda, k) * sum_{j in M(i)} e^{s'_ij - m'_i} v'_j
+ *                                   / sum_{j in M(i)} e^{s'_ij - m'_i}  +  R_i
+ * and O'_i = R_i when M(i) is empty.  Only the kept key blocks are visited.
+ * rho and r are the calibration's outputs (same layouts). */
+RT_API rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                         const rt_block_index* idx, const float* rho, const void* r,
+                         float lambda, int32_t step_distance, rt_ramp ramp, void* o, void* stream);
+
+/* Synchronises `stream`, returns the first device-side status recorded since
+ * the last call on the current device, and clears it. */
+RT_API rt_status rt_check_device_error(void* stream);
+
+/* Static string for a status code (never NULL). */
+RT_API const char* rt_status_string(rt_status s);
+
+/* Text of the last CUDA error seen by this library on this thread ("" if none). */
+RT_API const char* rt_last_cuda_error(void);
+
+/* Upper bound, in nanoseconds, on every mbarrier wait inside the kernels
+ * (default 4e9).  A wait that exceeds it records RT_ERR_TIMEOUT and the CTA
+ * drains its own in-flight copies and MMAs, frees its TMEM and returns.
+ * Process-wide; applies to launches made after the call.  0 restores the default. */
+RT_API rt_status rt_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Test hook for the bounded-wait path: launches one CTA that waits on an
+ * mbarrier no one arrives on, for at most limit_ns, then records
+ * RT_ERR_TIMEOUT.  Never faults or hangs. */
+RT_API rt_status rt_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Compute capability the library was built for (1000 = sm_100a). */
+RT_API int32_t rt_build_arch(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RT_B200_H */

@@ -1,0 +1,244 @@
+"""ctypes binding of the C ABI in ``include/rt.h`` (``librt_b200.so``).
+
+Argument marshalling only: the functions here carry the C entry points'
+names, check that tensors are CUDA tensors of the right dtype and layout,
+allocate outputs with torch when the caller gives none, and pass raw device
+pointers and the current CUDA stream.  Every step of the computation runs in
+the library's kernels.  There is no CPU fallback: without the built library
+or a CUDA device these functions raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librt_b200.so")
+
+RT_OK = 0
+RT_ERR_INVALID_ARGUMENT = 1
+RT_ERR_UNSUPPORTED = 2
+RT_ERR_CAPACITY = 3
+RT_ERR_CUDA = 4
+RT_ERR_TIMEOUT = 5
+RT_ERR_BAD_INDEX = 6
+
+RT_RAMP_MUL_LINEAR = 0
+RT_RAMP_ADD_LINEAR = 1
+RT_RAMP_GEOMETRIC = 2
+
+RT_BF16 = 0
+RT_F32 = 1
+
+EXPORTED = (
+    "rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_check_device_error",
+    "rt_status_string", "rt_last_cuda_error", "rt_set_wait_limit_ns", "rt_debug_wait_timeout",
+    "rt_build_arch",
+)
+
+
+class RtAttnDesc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+        ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64), ("stride_l", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_float), ("r_dtype", ctypes.c_int),
+    ]
+
+
+class RtBlockIndex(ctypes.Structure):
+    _fields_ = [
+        ("Hm", ctypes.c_int32), ("nqb", ctypes.c_int32), ("nkb", ctypes.c_int32),
+        ("nnz", ctypes.c_int64),
+        ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+    ]
+
+
+class RtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        lib = _lib
+        name = lib.rt_status_string(status).decode() if lib else str(status)
+        extra = lib.rt_last_cuda_error().decode() if (lib and status == RT_ERR_CUDA) else ""
+        super().__init__(f"{where}: {name}" + (f" ({extra})" if extra else ""))
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load librt_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m sparse_attention_diffusion_rt_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.rt_build_block_index.argtypes = [vp, i32, i32, i32, vp, vp, i64, ctypes.POINTER(i64), vp]
+    lib.rt_calibrate.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
+                                 vp, vp, vp, vp]
+    lib.rt_sparse_step.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
+                                   vp, vp, ctypes.c_float, i32, ctypes.c_int, vp, vp]
+    lib.rt_check_device_error.argtypes = [vp]
+    lib.rt_status_string.argtypes = [ctypes.c_int]
+    lib.rt_status_string.restype = ctypes.c_char_p
+    lib.rt_last_cuda_error.argtypes = []
+    lib.rt_last_cuda_error.restype = ctypes.c_char_p
+    lib.rt_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.rt_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.rt_build_arch.argtypes = []
+    for name in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_check_device_error",
+                 "rt_set_wait_limit_ns", "rt_debug_wait_timeout", "rt_build_arch"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _require_cuda(*tensors):
+    if not torch.cuda.is_available():
+        raise RuntimeError("librt_b200 needs a CUDA device; there is no CPU fallback")
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != RT_OK:
+        raise RtError(status, where)
+
+
+@dataclasses.dataclass
+class BlockIndex:
+    """CSR block index on the device (see rt_block_index in include/rt.h)."""
+    row_ptr: torch.Tensor      # int32 [Hm*nqb + 1]
+    col_idx: torch.Tensor      # int32 [nnz]
+    Hm: int
+    nqb: int
+    nkb: int
+    nnz: int
+
+    def as_c(self) -> RtBlockIndex:
+        return RtBlockIndex(self.Hm, self.nqb, self.nkb, self.nnz, self.row_ptr.data_ptr(),
+                            self.col_idx.data_ptr() if self.nnz > 0 else None)
+
+
+def rt_build_block_index(mask: torch.Tensor, stream=None) -> BlockIndex:
+    """Dense uint8 block mask [Hm, nqb, nkb] (CUDA) -> CSR BlockIndex."""
+    lib = load_library()
+    _require_cuda(mask)
+    if mask.dtype != torch.uint8 or mask.dim() != 3 or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous uint8 [Hm, nqb, nkb] tensor")
+    Hm, nqb, nkb = mask.shape
+    row_ptr = torch.empty(Hm * nqb + 1, dtype=torch.int32, device=mask.device)
+    cap = Hm * nqb * nkb
+    col = torch.empty(max(cap, 1), dtype=torch.int32, device=mask.device)
+    nnz = ctypes.c_int64(0)
+    _check(lib.rt_build_block_index(mask.data_ptr(), Hm, nqb, nkb, row_ptr.data_ptr(), col.data_ptr(),
+                                    cap, ctypes.byref(nnz), _stream_ptr(stream)),
+           "rt_build_block_index")
+    return BlockIndex(row_ptr, col[: nnz.value], Hm, nqb, nkb, nnz.value)
+
+
+def make_block_index(row_ptr: torch.Tensor, col_idx: torch.Tensor, Hm: int, nqb: int, nkb: int) -> BlockIndex:
+    """Wrap caller-made CSR arrays (CUDA int32) without validating them here;
+    the kernels validate every row they use and record RT_ERR_BAD_INDEX."""
+    return BlockIndex(row_ptr, col_idx, Hm, nqb, nkb, int(col_idx.numel()))
+
+
+def _desc(q: torch.Tensor, block: int, softmax_scale: float, r_dtype: torch.dtype) -> RtAttnDesc:
+    if q.dim() != 4 or q.stride(3) != 1:
+        raise ValueError("q/k/v/o/r must be [B, H, L, d] with d contiguous")
+    B, H, L, d = q.shape
+    sb, sh, sl, _ = q.stride()
+    rd = RT_F32 if r_dtype == torch.float32 else RT_BF16
+    return RtAttnDesc(B, H, L, d, block, sb, sh, sl, float(softmax_scale), rd)
+
+
+def _same_layout(ref: torch.Tensor, *ts):
+    for t in ts:
+        if t.shape != ref.shape or t.stride() != ref.stride():
+            raise ValueError("q, k, v, o and r must share shape and strides")
+
+
+def rt_calibrate(q, k, v, index: BlockIndex, *, block: int, o=None, rho=None, r=None,
+                 r_dtype=torch.bfloat16, softmax_scale: float = 0.0, stream=None):
+    """Calibration step: returns (O bf16, rho fp32 [B,H,L], R r_dtype)."""
+    lib = load_library()
+    _require_cuda(q, k, v, o, rho, r)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be bfloat16")
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    r = torch.empty_strided(q.shape, q.stride(), dtype=r_dtype, device=q.device) if r is None else r
+    rho = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if rho is None else rho
+    if o.dtype != torch.bfloat16 or r.dtype != r_dtype or rho.dtype != torch.float32 or not rho.is_contiguous():
+        raise ValueError("o must be bf16, r must be r_dtype, rho fp32 contiguous [B, H, L]")
+    _same_layout(q, k, v, o, r)
+    desc = _desc(q, block, softmax_scale, r_dtype)
+    idx = index.as_c()
+    _check(lib.rt_calibrate(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
+                            o.data_ptr(), rho.data_ptr(), r.data_ptr(), _stream_ptr(stream)),
+           "rt_calibrate")
+    return o, rho, r
+
+
+def rt_sparse_step(q, k, v, index: BlockIndex, rho, r, *, block: int, lam: float = 0.04,
+                   step_distance: int = 1, ramp: int = RT_RAMP_MUL_LINEAR, o=None,
+                   softmax_scale: float = 0.0, stream=None):
+    """Reshaped sparse step: returns O' (bf16)."""
+    lib = load_library()
+    _require_cuda(q, k, v, rho, r, o)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be bfloat16")
+    if r.dtype not in (torch.bfloat16, torch.float32) or rho.dtype != torch.float32 or not rho.is_contiguous():
+        raise ValueError("r must be bf16/fp32, rho fp32 contiguous [B, H, L]")
+    o = torch.empty_like(q) if o is None else o
+    if o.dtype != torch.bfloat16:
+        raise ValueError("o must be bfloat16")
+    _same_layout(q, k, v, o, r)
+    desc = _desc(q, block, softmax_scale, r.dtype)
+    idx = index.as_c()
+    _check(lib.rt_sparse_step(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
+                              rho.data_ptr(), r.data_ptr(), float(lam), int(step_distance), int(ramp),
+                              o.data_ptr(), _stream_ptr(stream)),
+           "rt_sparse_step")
+    return o
+
+
+def rt_check_device_error(stream=None) -> int:
+    """Synchronise, return and clear the first device-side status (0 = none)."""
+    lib = load_library()
+    _require_cuda()
+    return lib.rt_check_device_error(_stream_ptr(stream))
+
+
+def rt_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(load_library().rt_set_wait_limit_ns(int(limit_ns)), "rt_set_wait_limit_ns")
+
+
+def rt_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    lib = load_library()
+    _require_cuda()
+    _check(lib.rt_debug_wait_timeout(int(limit_ns), _stream_ptr(stream)), "rt_debug_wait_timeout")
+
+
+def rt_status_string(status: int) -> str:
+    return load_library().rt_status_string(int(status)).decode()
+
+
+def rt_build_arch() -> int:
+    return load_library().rt_build_arch()

@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI library (no GPU, no compute calls): it loads, it
+exports every entry point include/rt.h declares, the ctypes structures match
+the C layout, and host-side validation rejects bad arguments before any CUDA
+call is made."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_attention_diffusion_rt_b200 import build as rtbuild
+from sparse_attention_diffusion_rt_b200 import rt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rt.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rtbuild.build()
+    return rt.load_library()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"RT_API\s+[\w\s\*]+?\b(rt_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_check_device_error",
+              "rt_status_string"):
+        assert n in names
+    assert sorted(rt.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", rt.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, re.M))
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(lib, n)
+    assert {s for s in exported if s.startswith("rt_")} == set(_declared())
+
+
+def test_status_strings_and_arch(lib):
+    assert rt.rt_status_string(0) == "RT_OK"
+    assert rt.rt_status_string(6) == "RT_ERR_BAD_INDEX"
+    assert rt.rt_status_string(99) == "RT_ERR_UNKNOWN"
+    assert rt.rt_build_arch() == 1000
+
+
+def test_struct_layout_matches_c(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "rt.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(rt_attn_desc),"
+        " offsetof(rt_attn_desc, stride_b), offsetof(rt_attn_desc, softmax_scale), offsetof(rt_attn_desc, r_dtype),"
+        " sizeof(rt_block_index), offsetof(rt_block_index, nnz), offsetof(rt_block_index, col_idx));return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    got = list(map(int, subprocess.check_output([str(exe)]).split()))
+    want = [ctypes.sizeof(rt.RtAttnDesc), rt.RtAttnDesc.stride_b.offset, rt.RtAttnDesc.softmax_scale.offset,
+            rt.RtAttnDesc.r_dtype.offset, ctypes.sizeof(rt.RtBlockIndex), rt.RtBlockIndex.nnz.offset,
+            rt.RtBlockIndex.col_idx.offset]
+    assert got == want
+
+
+def test_host_validation_without_gpu(lib):
+    """Argument errors are returned before any CUDA call (safe without a device)."""
+    vp = ctypes.c_void_p
+    assert lib.rt_calibrate(None, vp(16), vp(16), vp(16), None, vp(16), vp(16), vp(16), None) == rt.RT_ERR_INVALID_ARGUMENT
+    desc = rt.RtAttnDesc(1, 1, 128, 64, 128, 8192, 8192, 64, 0.0, 0)
+    idx = rt.RtBlockIndex(1, 1, 1, 1, 4096, 4096)
+    args = (vp(4096), vp(4096), vp(4096), ctypes.byref(idx), vp(4096), vp(4096), vp(4096), None)
+    bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)          # d % 8 != 0
+    assert lib.rt_calibrate(ctypes.byref(bad), *args) == rt.RT_ERR_UNSUPPORTED
+    bad = rt.RtAttnDesc(1, 1, 128, 64, 32, 8192, 8192, 64, 0.0, 0)           # block 32
+    assert lib.rt_calibrate(ctypes.byref(bad), *args) == rt.RT_ERR_UNSUPPORTED
+    bad = rt.RtAttnDesc(1, 1, 128, 64, 128, 8192, 8192, 64, -1.0, 0)         # negative scale
+    assert lib.rt_calibrate(ctypes.byref(bad), *args) == rt.RT_ERR_INVALID_ARGUMENT
+    mis = (vp(4096 + 8),) + args[1:]                                          # misaligned q
+    assert lib.rt_calibrate(ctypes.byref(desc), *mis) == rt.RT_ERR_INVALID_ARGUMENT
+    idx2 = rt.RtBlockIndex(1, 2, 2, 1, 4096, 4096)                           # nqb != ceil(L/block)
+    assert lib.rt_calibrate(ctypes.byref(desc), vp(4096), vp(4096), vp(4096), ctypes.byref(idx2), vp(4096),
+                            vp(4096), vp(4096), None) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_sparse_step(ctypes.byref(desc), *args[:4], vp(4096), vp(4096), ctypes.c_float(0.04), 1, 7,
+                              vp(4096), None) == rt.RT_ERR_INVALID_ARGUMENT     # unknown ramp
+    assert lib.rt_sparse_step(ctypes.byref(desc), *args[:4], vp(4096), vp(4096), ctypes.c_float(0.04), -1, 0,
+                              vp(4096), None) == rt.RT_ERR_INVALID_ARGUMENT     # negative step distance
+    nnz = ctypes.c_int64(0)
+    assert lib.rt_build_block_index(None, 1, 1, 1, vp(16), vp(16), 1, ctypes.byref(nnz), None) == \
+        rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_build_block_index(vp(16), 1, 0, 1, vp(16), vp(16), 1, ctypes.byref(nnz), None) == \
+        rt.RT_ERR_INVALID_ARGUMENT
+
+
+def test_binding_refuses_without_cuda(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("CUDA present")
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        rt.rt_calibrate(q, q, q, None, block=128)

@@ -1,0 +1,312 @@
+"""GPU parity: the C-ABI kernels against the float64 CPU oracle, element by
+element, on identical seeded bf16 inputs.
+
+Sizes the oracle finishes in seconds are checked in full (several tiles and a
+ragged tail); the full-size CogVideoX-like and long-video workloads, launched
+exactly as bench.py launches them, are checked on sampled rows.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import check_out, check_rho, f64
+from oracle import reference as ref
+from sparse_attention_diffusion_rt_b200 import inputs
+from sparse_attention_diffusion_rt_b200 import rt
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _index(mask_np):
+    return rt.rt_build_block_index(torch.from_numpy(np.ascontiguousarray(mask_np)).to(DEV))
+
+
+def _ok():
+    st = rt.rt_check_device_error()
+    assert st == rt.RT_OK, rt.rt_status_string(st)
+
+
+def _stats_inputs(shape, seed, r_dtype=torch.bfloat16):
+    """Synthetic cached statistics for isolated sparse-step parity (not from the CUDA path)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    B, H, L, d = shape
+    rho = torch.rand((B, H, L), generator=g, dtype=torch.float32)
+    r = (0.1 * torch.randn(shape, generator=g, dtype=torch.float32)).to(r_dtype)
+    return rho.to(DEV), r.to(DEV)
+
+
+# ---------------------------------------------------------------------------
+# block index
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(inputs.WORKLOADS))
+def test_block_index_workload_masks_bit_exact(name):
+    mask = inputs.block_mask(inputs.WORKLOADS[name])
+    idx = _index(mask)
+    rp, ci = ref.build_block_index_ref(mask)
+    assert idx.nnz == len(ci)
+    np.testing.assert_array_equal(idx.row_ptr.cpu().numpy(), rp)
+    np.testing.assert_array_equal(idx.col_idx.cpu().numpy(), ci)
+
+
+@pytest.mark.parametrize("Hm,nqb,nkb,dens,seed", [(1, 1, 1, 1.0, 0), (3, 17, 33, 0.2, 1), (2, 50, 70, 0.0, 2),
+                                                   (4, 300, 300, 0.05, 3), (1, 1100, 1000, 0.5, 4),
+                                                   (2, 7, 1, 0.5, 5)])
+def test_block_index_random_bit_exact(Hm, nqb, nkb, dens, seed):
+    mask = inputs.random_block_mask(Hm, nqb, nkb, dens, seed)
+    idx = _index(mask)
+    rp, ci = ref.build_block_index_ref(mask)
+    np.testing.assert_array_equal(idx.row_ptr.cpu().numpy(), rp)
+    np.testing.assert_array_equal(idx.col_idx.cpu().numpy(), ci)
+
+
+def test_block_index_capacity_error():
+    mask = torch.ones((1, 4, 4), dtype=torch.uint8, device=DEV)
+    row_ptr = torch.empty(5, dtype=torch.int32, device=DEV)
+    col = torch.full((10,), -7, dtype=torch.int32, device=DEV)
+    lib = rt.load_library()
+    import ctypes
+    nnz = ctypes.c_int64(0)
+    st = lib.rt_build_block_index(mask.data_ptr(), 1, 4, 4, row_ptr.data_ptr(), col.data_ptr(), 10,
+                                  ctypes.byref(nnz), rt._stream_ptr(None))
+    assert st == rt.RT_ERR_CAPACITY and nnz.value == 16
+    assert row_ptr.cpu().tolist() == [0, 4, 8, 12, 16]
+    assert col.cpu().tolist() == [0, 1, 2, 3] * 2 + [0, 1]      # only positions that fit
+
+
+# ---------------------------------------------------------------------------
+# small problems, full tensors
+# ---------------------------------------------------------------------------
+
+def _run_cycle_full(q, k, v, q2, k2, v2, mask, block, lam=0.04, kdist=1, ramp=rt.RT_RAMP_MUL_LINEAR,
+                    r_dtype=torch.bfloat16, scale=0.0, Hm_mask=None):
+    idx = _index(mask)
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=block, r_dtype=r_dtype, softmax_scale=scale)
+    o2 = rt.rt_sparse_step(q2, k2, v2, idx, rho, r, block=block, lam=lam, step_distance=kdist, ramp=ramp,
+                           softmax_scale=scale)
+    torch.cuda.synchronize()
+    _ok()
+    sc = scale if scale else None
+    O, RHO, R = ref.calibrate_ref(f64(q), f64(k), f64(v), mask, block, scale=sc)
+    check_out(f64(o), O, "calibrate O")
+    check_out(f64(r), R, "calibrate R")
+    check_rho(f64(rho), RHO)
+    O2 = ref.sparse_step_ref(f64(q2), f64(k2), f64(v2), mask, block, RHO, R, lam, kdist, ramp, scale=sc)
+    check_out(f64(o2), O2, "sparse O (end to end)")
+    # isolated sparse step on synthetic statistics
+    rho_s, r_s = _stats_inputs(tuple(q.shape), 99, r_dtype)
+    o3 = rt.rt_sparse_step(q2, k2, v2, idx, rho_s, r_s, block=block, lam=lam, step_distance=kdist, ramp=ramp,
+                           softmax_scale=scale)
+    torch.cuda.synchronize()
+    _ok()
+    O3 = ref.sparse_step_ref(f64(q2), f64(k2), f64(v2), mask, block, f64(rho_s), f64(r_s), lam, kdist, ramp,
+                             scale=sc)
+    check_out(f64(o3), O3, "sparse O (isolated)")
+
+
+@pytest.mark.parametrize("name", ["tiny", "pixart", "hunyuan"])
+def test_workload_cycle_full(name):
+    w = inputs.WORKLOADS[name]
+    steps = inputs.qkv_steps(w, 2, device=DEV)
+    mask = inputs.block_mask(w)
+    _run_cycle_full(*steps[0], *steps[1], mask, w.block, lam=w.lam, kdist=1)
+
+
+@pytest.mark.parametrize("d", [16, 32, 48, 64, 72, 88, 96, 104, 120, 128])
+def test_head_dims_ragged_tail(d):
+    B, H, L, blk = 1, 2, 300, 128              # 3 query blocks, tail of 44
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=d, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=1000 + d, device=DEV)
+    mask = inputs.random_block_mask(1, 3, 3, 0.5, seed=d, ensure_nonempty=True)
+    _run_cycle_full(q, k, v, q2, k2, v2, mask, blk)
+
+
+@pytest.mark.parametrize("ramp", [rt.RT_RAMP_MUL_LINEAR, rt.RT_RAMP_ADD_LINEAR, rt.RT_RAMP_GEOMETRIC])
+def test_ramp_modes_and_fp32_residual(ramp):
+    B, H, L, d, blk = 2, 3, 520, 64, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=5, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=6, device=DEV)
+    mask = inputs.random_block_mask(H, 5, 5, 0.4, seed=7)           # per-head masks, some empty rows
+    _run_cycle_full(q, k, v, q2, k2, v2, mask, blk, lam=0.04, kdist=3, ramp=ramp, r_dtype=torch.float32)
+
+
+@pytest.mark.parametrize("d", [72, 88, 128])
+def test_fp32_residual_padded_dims(d):
+    B, H, L, blk = 1, 2, 400, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=11, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=12, device=DEV)
+    mask = inputs.random_block_mask(1, 4, 4, 0.5, seed=13, ensure_nonempty=True)
+    _run_cycle_full(q, k, v, q2, k2, v2, mask, blk, r_dtype=torch.float32)
+
+
+def test_block64_and_scale_override():
+    B, H, L, d, blk = 1, 2, 200, 64, 64        # 4 query blocks of 64, tail of 8
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=21, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=22, device=DEV)
+    mask = inputs.random_block_mask(1, 4, 4, 0.5, seed=23)
+    _run_cycle_full(q, k, v, q2, k2, v2, mask, blk, scale=0.1)
+
+
+def test_dense_and_empty_masks():
+    B, H, L, d, blk = 1, 2, 384, 64, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=31, device=DEV)
+    dense = np.ones((1, 3, 3), dtype=np.uint8)
+    idx = _index(dense)
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=blk)
+    torch.cuda.synchronize()
+    _ok()
+    assert torch.all(rho == 1.0)
+    assert torch.all(r == 0)
+    o_full = ref.full_attention_ref(f64(q), f64(k), f64(v))
+    check_out(f64(o), o_full, "dense calibrate O")
+    empty = np.zeros((1, 3, 3), dtype=np.uint8)
+    idx0 = _index(empty)
+    assert idx0.nnz == 0
+    o, rho, r = rt.rt_calibrate(q, k, v, idx0, block=blk)
+    torch.cuda.synchronize()
+    _ok()
+    assert torch.all(rho == 0.0)
+    check_out(f64(r), o_full, "empty-mask R is the full output")
+    rho_s, r_s = _stats_inputs((B, H, L, d), 5)
+    o2 = rt.rt_sparse_step(q, k, v, idx0, rho_s, r_s, block=blk)
+    torch.cuda.synchronize()
+    _ok()
+    assert torch.equal(o2, r_s)                # empty kept set: O' = R exactly
+
+
+def test_invariant_same_inputs_lambda0_gives_full_attention():
+    w = inputs.WORKLOADS["pixart"]
+    q, k, v = inputs.initial_qkv(w, device=DEV)
+    idx = _index(inputs.block_mask(w))
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=w.block, r_dtype=torch.float32)
+    o2 = rt.rt_sparse_step(q, k, v, idx, rho, r, block=w.block, lam=0.0, step_distance=1)
+    torch.cuda.synchronize()
+    _ok()
+    full = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float())
+    check_out(f64(o2), f64(full), "sparse(lambda=0) vs full attention")
+    check_out(f64(o), f64(full), "calibrate O vs full attention")
+
+
+def test_strided_layout_bsHd():
+    """[B, L, H, d] storage viewed as [B, H, L, d] (non-contiguous strides)."""
+    B, H, L, d, blk = 2, 4, 256, 64, 128
+    g = torch.Generator(device=DEV).manual_seed(41)
+    base = [torch.randn((B, L, H, d), generator=g, device=DEV).to(torch.bfloat16) for _ in range(6)]
+    q, k, v, q2, k2, v2 = (t.permute(0, 2, 1, 3) for t in base)
+    mask = inputs.random_block_mask(1, 2, 2, 0.5, seed=42, ensure_nonempty=True)
+    idx = _index(mask)
+    o = torch.empty_like(base[0]).permute(0, 2, 1, 3)
+    r = torch.empty_like(base[0]).permute(0, 2, 1, 3)
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=blk, o=o, r=r)
+    o2 = torch.empty_like(base[0]).permute(0, 2, 1, 3)
+    o2 = rt.rt_sparse_step(q2, k2, v2, idx, rho, r, block=blk, o=o2)
+    torch.cuda.synchronize()
+    _ok()
+    O, RHO, R = ref.calibrate_ref(f64(q), f64(k), f64(v), mask, blk)
+    check_out(f64(o), O, "strided O")
+    check_out(f64(r), R, "strided R")
+    check_rho(f64(rho), RHO)
+    O2 = ref.sparse_step_ref(f64(q2), f64(k2), f64(v2), mask, blk, RHO, R, 0.04, 1)
+    check_out(f64(o2), O2, "strided sparse O")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled rows (launched as bench.py launches them)
+# ---------------------------------------------------------------------------
+
+def _sample_rows(L, block, rng, n_mid=6):
+    nqb = -(-L // block)
+    blocks = sorted(set([0, 1, nqb - 1] + list(rng.integers(0, nqb, n_mid))))
+    rows = []
+    for qb in blocks:
+        lo, hi = qb * block, min(L, (qb + 1) * block)
+        rows += [lo, hi - 1, int(rng.integers(lo, hi))]
+    return np.array(sorted(set(rows)))
+
+
+@pytest.mark.parametrize("name", ["cogvideox", "longvideo-3.1", "longvideo-25"])
+def test_full_size_sampled_rows(name):
+    w = inputs.WORKLOADS[name]
+    steps = inputs.qkv_steps(w, 2, device=DEV)
+    mask = inputs.block_mask(w)
+    idx = _index(mask)
+    (q, k, v), (q2, k2, v2) = steps
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=w.block)
+    o2 = rt.rt_sparse_step(q2, k2, v2, idx, rho, r, block=w.block, lam=w.lam, step_distance=1)
+    torch.cuda.synchronize()
+    _ok()
+    rng = np.random.default_rng(w.seed)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (0, int(rng.integers(w.H)))]
+    for b, h in heads:
+        rows = _sample_rows(w.L, w.block, rng)
+        qf, kf, vf = f64(q[b, h]), f64(k[b, h]), f64(v[b, h])
+        O, RHO, R = ref.calibrate_rows_ref(qf, kf, vf, mask[0], w.block, rows)
+        check_out(f64(o[b, h, rows]), O, f"{name} calibrate O (b{b} h{h})")
+        check_out(f64(r[b, h, rows]), R, f"{name} calibrate R (b{b} h{h})")
+        check_rho(f64(rho[b, h, rows]), RHO, f"{name} rho")
+        O2 = ref.sparse_step_rows_ref(f64(q2[b, h]), f64(k2[b, h]), f64(v2[b, h]), mask[0], w.block, rows,
+                                      RHO, R, w.lam, 1)
+        check_out(f64(o2[b, h, rows]), O2, f"{name} sparse O (b{b} h{h})")
+    # properties that hold at any size
+    assert torch.all(torch.isfinite(o.float())) and torch.all(torch.isfinite(o2.float()))
+    assert torch.all((rho >= 0) & (rho <= 1.0 + 1e-6))
+    del steps, q, k, v, q2, k2, v2, o, o2, r, rho
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# device-side error paths (never fault: bad index is detected and recorded)
+# ---------------------------------------------------------------------------
+
+def _bad_index_run(row_ptr, col_idx, nqb):
+    B, H, L, d, blk = 1, 2, nqb * 128, 64, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=3, device=DEV)
+    idx = rt.make_block_index(torch.tensor(row_ptr, dtype=torch.int32, device=DEV),
+                              torch.tensor(col_idx, dtype=torch.int32, device=DEV), 1, nqb, nqb)
+    rt.rt_calibrate(q, k, v, idx, block=blk)
+    return rt.rt_check_device_error()
+
+
+def test_bad_col_idx_out_of_range_recorded():
+    assert _bad_index_run([0, 1, 2], [0, 5], 2) == rt.RT_ERR_BAD_INDEX
+    assert rt.rt_check_device_error() == rt.RT_OK            # cleared
+
+
+def test_bad_col_idx_not_ascending_recorded():
+    assert _bad_index_run([0, 2, 3], [1, 0, 1], 2) == rt.RT_ERR_BAD_INDEX
+
+
+def test_bad_row_ptr_recorded():
+    assert _bad_index_run([0, 3, 2], [0, 1], 2) == rt.RT_ERR_BAD_INDEX
+
+
+def test_good_index_after_errors_still_correct():
+    test_workload_cycle_full("tiny")
+
+
+def test_bounded_wait_reports_timeout():
+    rt.rt_debug_wait_timeout(2_000_000)                     # 2 ms on a barrier nobody completes
+    assert rt.rt_check_device_error() == rt.RT_ERR_TIMEOUT
+    assert rt.rt_check_device_error() == rt.RT_OK
+
+
+def test_host_validation_rejects_before_launch():
+    q, k, v = inputs.random_qkv(1, 1, 128, 64, seed=0, device=DEV)
+    idx = _index(np.ones((1, 1, 1), dtype=np.uint8))
+    with pytest.raises(rt.RtError) as e:
+        rt.rt_calibrate(q, k, v, idx, block=32)
+    assert e.value.status == rt.RT_ERR_UNSUPPORTED
+    q20, k20, v20 = inputs.random_qkv(1, 1, 128, 20, seed=0, device=DEV)
+    with pytest.raises(rt.RtError) as e:
+        rt.rt_calibrate(q20, k20, v20, idx, block=128)
+    assert e.value.status == rt.RT_ERR_UNSUPPORTED
+    bad_idx = rt.BlockIndex(idx.row_ptr, idx.col_idx, 1, 2, 2, idx.nnz)      # nqb inconsistent with L
+    with pytest.raises(rt.RtError) as e:
+        rt.rt_calibrate(q, k, v, bad_idx, block=128)
+    assert e.value.status == rt.RT_ERR_INVALID_ARGUMENT
+    _ok()
