@@ -22,6 +22,7 @@ Multi-GPU (weak scaling, independent replicas, no data-path collective):
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -250,6 +251,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     rt.load_library()
     w = inputs.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-h{args.heads}")
     peaks = load_peaks()
     n_steps = 1 + w.n_sparse_steps
     qkv = inputs.qkv_steps(w, n_steps, device=dev)
@@ -396,6 +399,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (a smaller case for profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

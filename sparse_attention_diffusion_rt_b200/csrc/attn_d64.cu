@@ -4,12 +4,12 @@
 namespace rtb {
 
 cudaError_t launch_attn_d64(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                           int smem, cudaStream_t s) {
-  if (block == 64) return cal ? launch_attn_impl<64, 64, true>(tm, p, grid, smem, s)
-                            : launch_attn_impl<64, 64, false>(tm, p, grid, smem, s);
+                           cudaStream_t s) {
+  if (block == 64) return cal ? launch_attn_impl<64, 64, true>(tm, p, grid, s)
+                            : launch_attn_impl<64, 64, false>(tm, p, grid, s);
   if (block != 128) return cudaErrorInvalidValue;
-  return cal ? launch_attn_impl<64, 128, true>(tm, p, grid, smem, s)
-             : launch_attn_impl<64, 128, false>(tm, p, grid, smem, s);
+  return cal ? launch_attn_impl<64, 128, true>(tm, p, grid, s)
+             : launch_attn_impl<64, 128, false>(tm, p, grid, s);
 }
 
 }  // namespace rtb

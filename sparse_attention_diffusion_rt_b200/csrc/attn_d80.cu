@@ -4,10 +4,10 @@
 namespace rtb {
 
 cudaError_t launch_attn_d80(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                           int smem, cudaStream_t s) {
+                           cudaStream_t s) {
   if (block != 128) return cudaErrorInvalidValue;
-  return cal ? launch_attn_impl<80, 128, true>(tm, p, grid, smem, s)
-             : launch_attn_impl<80, 128, false>(tm, p, grid, smem, s);
+  return cal ? launch_attn_impl<80, 128, true>(tm, p, grid, s)
+             : launch_attn_impl<80, 128, false>(tm, p, grid, s);
 }
 
 }  // namespace rtb

@@ -13,23 +13,31 @@ namespace rtb {
 // share an SM (each allocates all 512 TMEM columns).
 constexpr int kMinSmem = 120 * 1024;
 
-// Dynamic shared memory the launch needs (bytes).
-int attn_smem_bytes(int dpad, bool cal, bool r_f32);
+// Dynamic shared memory one launch of attn_kernel<DPAD, BN, CAL> needs (bytes),
+// never below kMinSmem.
+template <int DPAD, int BN>
+constexpr int attn_smem_bytes(bool cal, bool r_f32) {
+  using C = Cfg<DPAD, BN>;
+  const int need = cal ? C::SMEM_CAL : C::OFF_R + (r_f32 ? C::R_MAX_BYTES : C::Q_BYTES) + 1024;
+  return need > kMinSmem ? need : kMinSmem;
+}
 
 // Launch the attention kernel instantiated for (dpad, block, cal).
 // Returns cudaErrorInvalidValue for an instantiation that does not exist.
 cudaError_t launch_attn_d64(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                            int smem, cudaStream_t s);
+                            cudaStream_t s);
 cudaError_t launch_attn_d80(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                            int smem, cudaStream_t s);
+                            cudaStream_t s);
 cudaError_t launch_attn_d96(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                            int smem, cudaStream_t s);
+                            cudaStream_t s);
 cudaError_t launch_attn_d128(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
-                             int smem, cudaStream_t s);
+                             cudaStream_t s);
 
 template <int DPAD, int BN, bool CAL>
-cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, int smem,
-                             cudaStream_t s) {
+cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, cudaStream_t s) {
+  constexpr int kMaxSmem = attn_smem_bytes<DPAD, BN>(CAL, true) > attn_smem_bytes<DPAD, BN>(CAL, false)
+                               ? attn_smem_bytes<DPAD, BN>(CAL, true) : attn_smem_bytes<DPAD, BN>(CAL, false);
+  const int smem = attn_smem_bytes<DPAD, BN>(CAL, p.r_f32 != 0);
   auto kern = attn_kernel<DPAD, BN, CAL>;
   // the shared-memory opt-in is a per-device function attribute: set it once per device
   static std::atomic<unsigned long long> configured{0};
@@ -38,8 +46,7 @@ cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, i
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg<DPAD, BN>::SMEM_SPARSE > kMinSmem ? Cfg<DPAD, BN>::SMEM_SPARSE : kMinSmem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }

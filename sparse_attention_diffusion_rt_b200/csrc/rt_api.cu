@@ -168,20 +168,12 @@ rt_status fill_common(const rt_attn_desc& d, const rt_block_index& idx, AttnPara
 cudaError_t dispatch(int dpad, bool cal, const rt_attn_desc& d, const TmaSet& tm, const AttnParams& p,
                      cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(p.nqb), static_cast<unsigned>(d.H), static_cast<unsigned>(d.B));
-  const int smem = attn_smem_bytes(dpad, cal, d.r_dtype == RT_F32);
   switch (dpad) {
-    case 64: return launch_attn_d64(cal, d.block, tm, p, grid, smem, s);
-    case 80: return launch_attn_d80(cal, d.block, tm, p, grid, smem, s);
-    case 96: return launch_attn_d96(cal, d.block, tm, p, grid, smem, s);
-    default: return launch_attn_d128(cal, d.block, tm, p, grid, smem, s);
+    case 64: return launch_attn_d64(cal, d.block, tm, p, grid, s);
+    case 80: return launch_attn_d80(cal, d.block, tm, p, grid, s);
+    case 96: return launch_attn_d96(cal, d.block, tm, p, grid, s);
+    default: return launch_attn_d128(cal, d.block, tm, p, grid, s);
   }
-}
-
-template <int DPAD>
-int smem_for(bool cal, bool r_f32) {
-  using C = Cfg<DPAD, 128>;
-  const int need = cal ? C::SMEM_CAL : C::OFF_R + (r_f32 ? C::R_MAX_BYTES : C::Q_BYTES) + 1024;
-  return need > kMinSmem ? need : kMinSmem;
 }
 
 __global__ void debug_wait_kernel(unsigned long long limit_ns, unsigned int* status) {
@@ -203,17 +195,6 @@ __global__ void debug_wait_kernel(unsigned long long limit_ns, unsigned int* sta
 }
 
 }  // namespace
-
-namespace rtb {
-int attn_smem_bytes(int dpad, bool cal, bool r_f32) {
-  switch (dpad) {
-    case 64: return smem_for<64>(cal, r_f32);
-    case 80: return smem_for<80>(cal, r_f32);
-    case 96: return smem_for<96>(cal, r_f32);
-    default: return smem_for<128>(cal, r_f32);
-  }
-}
-}  // namespace rtb
 
 extern "C" {
 
