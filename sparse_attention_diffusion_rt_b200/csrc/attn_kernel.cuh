@@ -34,6 +34,7 @@
 
 #include "ptx.cuh"
 #include "rt.h"
+#include "softmax.cuh"
 
 namespace rtb {
 
@@ -61,6 +62,8 @@ struct AttnParams {
   const int* col_idx;
   float scale_log2;        // softmax scale * log2(e)
   const float* rho_in;     // sparse step
+  const void* r_in;        // sparse step residual (read directly when fp32)
+  long long stride_b, stride_h, stride_l;
   float ramp_mul, ramp_add;
   float* rho_out;          // calibration
   int r_f32;
@@ -293,21 +296,6 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Ctrl& ctl, uint8_t
   }
 }
 
-// Rescale one TMEM accumulator row (this thread's lane) by alpha.
-template <int DPAD>
-__device__ __forceinline__ void rescale_row(uint32_t taddr, float alpha) {
-#pragma unroll
-  for (int c = 0; c < DPAD; c += 16) {
-    uint32_t r[16];
-    tmem_ld_x16(taddr + c, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-    tmem_st_x16(taddr + c, r);
-  }
-  tmem_wait_st();
-}
-
 // Residual row chunk (16 columns starting at c) from a bf16 or fp32 tile in the
 // chunked, swizzled shared-memory layout the TMA copies use.
 template <int DPAD>
@@ -393,23 +381,14 @@ __device__ __forceinline__ void softmax_role(const TmaSet& tm, const AttnParams&
     if (!ok) break;
     tc_fence_after();
     uint32_t s[BN];
-#pragma unroll
-    for (int c = 0; c < BN; c += 32) tmem_ld_x32(tS + c, *reinterpret_cast<uint32_t(*)[32]>(&s[c]));
+    load_scores<BN>(tS, s);
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(&ctl.s_free);
 
     const int kb = CAL ? j : __ldg(p.col_idx + ctl.row_start + j);
-    const int valid = p.L - kb * BN;                 // keys of this block inside the sequence
-    if (valid < BN) {
-#pragma unroll
-      for (int c = 0; c < BN; ++c)
-        if (c >= valid) s[c] = __float_as_uint(-INFINITY);
-    }
-    float mx = __uint_as_float(s[0]);
-#pragma unroll
-    for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-    mx *= sl2;
+    mask_tail<BN>(s, p.L - kb * BN);                 // keys past the end of the sequence
+    const float mx = row_max<BN>(s) * sl2;
     if (j == 0) {
       m = mx;
     } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
@@ -426,20 +405,8 @@ __device__ __forceinline__ void softmax_role(const TmaSet& tm, const AttnParams&
       if (CAL && any_out) rescale_row<DPAD>(tOut, alpha);
       m = m_new;
     }
-    float sum = 0.f;
     const uint32_t tP = tmem + lane_base + ((j & 1) ? C::T_P1 : C::T_P0);
-#pragma unroll
-    for (int c0 = 0; c0 < BN; c0 += 64) {
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c]), sl2, -m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c + 1]), sl2, -m));
-        sum += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      tmem_st_x32(tP + c0 / 2, pk);
-    }
+    const float sum = exp_pack_store<BN>(s, sl2, m, tP);
     if (CAL) {
       if (is_kept(ctl, kb)) { l += sum; any_in = true; } else { l_out += sum; any_out = true; }
     } else {

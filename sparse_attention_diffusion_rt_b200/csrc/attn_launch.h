@@ -6,6 +6,7 @@
 #include <atomic>
 
 #include "attn_kernel.cuh"
+#include "sparse_kernel.cuh"
 
 namespace rtb {
 
@@ -51,6 +52,30 @@ cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, c
     configured.fetch_or(bit);
   }
   kern<<<grid, kThreads, smem, s>>>(tm, p);
+  return cudaGetLastError();
+}
+
+// Persistent sparse-step kernel (128-token blocks): one CTA per SM.
+template <int DPAD>
+cudaError_t launch_sparse_impl(const TmaSet& tm, const AttnParams& p, cudaStream_t s) {
+  auto kern = sparse_kernel<DPAD>;
+  constexpr int smem = SpCfg<DPAD>::SMEM > kMinSmem ? SpCfg<DPAD>::SMEM : kMinSmem;
+  static std::atomic<unsigned long long> configured{0};
+  static int sm_count[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sm_count[dev & 63], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const long long ntiles = static_cast<long long>(p.B) * p.H * p.nqb;
+  const int grid = static_cast<int>(ntiles < sm_count[dev & 63] ? ntiles : sm_count[dev & 63]);
+  kern<<<grid, kThreads, smem, s>>>(tm, p, static_cast<int>(ntiles));
   return cudaGetLastError();
 }
 

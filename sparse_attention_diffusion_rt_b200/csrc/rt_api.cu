@@ -280,6 +280,10 @@ rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k,
   AttnParams p;
   if ((st = fill_common(d, *idx, p)) != RT_OK) return st;
   p.rho_in = rho;
+  p.r_in = r;
+  p.stride_b = d.stride_b;
+  p.stride_h = d.stride_h;
+  p.stride_l = d.stride_l;
   p.ramp_mul = static_cast<float>(mul);
   p.ramp_add = static_cast<float>(add);
   TmaSet tm;

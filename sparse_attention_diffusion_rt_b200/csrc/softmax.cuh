@@ -1,0 +1,88 @@
+// Row-wise pieces of the online softmax shared by the calibration and sparse
+// kernels.  Thread t owns query row t of the tile (TMEM lane t), so row
+// reductions are in-thread; they are written as 8 independent chains so that
+// one warp per scheduler keeps the FMNMX/FADD pipes and the MUFU busy instead
+// of waiting on a serial dependency.
+#pragma once
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace rtb {
+
+template <int BN>
+__device__ __forceinline__ float row_max(const uint32_t (&s)[BN]) {
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
+#pragma unroll
+  for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+  return mx[0];
+}
+
+// Set logits of key columns >= valid (keys past the end of the sequence) to -inf.
+template <int BN>
+__device__ __forceinline__ void mask_tail(uint32_t (&s)[BN], int valid) {
+  if (valid < BN) {
+#pragma unroll
+    for (int c = 0; c < BN; ++c)
+      if (c >= valid) s[c] = __float_as_uint(-INFINITY);
+  }
+}
+
+// p_c = 2^(s_c * sl2 - m) for the whole row block; P is stored as bf16 pairs
+// into TMEM columns [tP, tP + BN/2) of this thread's lane.  Returns sum_c p_c
+// (of the fp32 values).  The caller waits for the stores (tmem_wait_st).
+template <int BN>
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BN], float sl2, float m, uint32_t tP) {
+  float sum[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum[i] = 0.f;
+  const float neg_m = -m;
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c]), sl2, neg_m));
+      const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c + 1]), sl2, neg_m));
+      sum[(2 * c) & 7] += p0;
+      sum[(2 * c + 1) & 7] += p1;
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_x32(tP + c0 / 2, pk);
+  }
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) sum[i] += sum[i + w];
+  return sum[0];
+}
+
+// Load BN fp32 logits of this thread's row from TMEM (caller waits with tmem_wait_ld).
+template <int BN>
+__device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[BN]) {
+#pragma unroll
+  for (int c = 0; c < BN; c += 32) tmem_ld_x32(tS + c, *reinterpret_cast<uint32_t(*)[32]>(&s[c]));
+}
+
+// Rescale one TMEM accumulator row (this thread's lane) by alpha.
+template <int DPAD>
+__device__ __forceinline__ void rescale_row(uint32_t taddr, float alpha) {
+#pragma unroll
+  for (int c = 0; c < DPAD; c += 16) {
+    uint32_t r[16];
+    tmem_ld_x16(taddr + c, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+    tmem_st_x16(taddr + c, r);
+  }
+  tmem_wait_st();
+}
+
+}  // namespace rtb

@@ -1,0 +1,477 @@
+// Persistent sm_100a kernel for Re-ttention's reshaped sparse step,
+//   O'_i = rho_hat_i * softmax over the kept key blocks (s'_i) . v'  +  R_i
+// (O'_i = R_i for a query block with no kept key block), with
+// rho_hat = min(1, rho * ramp_mul + ramp_add)  ("Re-ttention", OpenReview
+// replies to W1: the sparse softmax rescaled by the cached denominator ratio,
+// plus the cached residual of the masked tokens; reply to Pwod's W1: ramp-up).
+//
+// One CTA per SM walks the (batch, head, query block) tiles tile = blockIdx.x
+// + i * gridDim.x, query block fastest so that concurrent CTAs share the
+// head's K/V in L2.  Roles (192 threads):
+//   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
+//   warp 4     producer: validates each tile's CSR row (all lanes), then lane 0
+//              issues the TMA loads: Q (double-buffered for d <= 96), the kept
+//              K/V blocks through an NST-stage ring, and the residual tile
+//   warp 5     lane 0 issues the tcgen05 MMAs: S = Q K^T into TMEM, O += P V
+//              with P read from TMEM
+// Tile metadata flows through a 2-slot ring (ti_*).  Every per-block barrier
+// phase is indexed by a block counter that runs across tiles, so the MMA warp
+// starts the next tile's QK^T while the softmax warps finish the previous
+// tile's epilogue; the output leaves through a shared-memory staging tile and
+// a TMA store that is only waited for when its staging slot comes round again.
+//
+// TMEM columns: S [0,128) fp32 logits, P0/P1 [128,256) bf16 probabilities,
+// O [256, 256+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
+// and every role drains what it has in flight before TMEM is freed.
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+
+#include "attn_kernel.cuh"
+#include "ptx.cuh"
+#include "softmax.cuh"
+
+namespace rtb {
+
+template <int DPAD>
+struct SpCfg {
+  static constexpr int BN = 128;
+  static constexpr int C1 = DPAD - 64;
+  static constexpr int C1B = C1 * 2;
+  static constexpr uint32_t C1SWZ = C1 == 16 ? SWZ_32B : (C1 == 32 ? SWZ_64B : SWZ_128B);
+  static constexpr int QBUF = DPAD <= 96 ? 2 : 1;
+  static constexpr int NST = DPAD <= 80 ? 3 : 2;
+  static constexpr int OSTG = DPAD <= 96 ? 2 : 1;
+  static constexpr int TILE_BYTES = 128 * DPAD * 2;          // one bf16 [128][DPAD] tile
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;          // K + V
+  static constexpr int OFF_Q = 1024;
+  static constexpr int OFF_STAGE = OFF_Q + QBUF * TILE_BYTES;
+  static constexpr int OFF_R = OFF_STAGE + NST * STAGE_BYTES;
+  static constexpr int OFF_OST = OFF_R + TILE_BYTES;
+  static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+  static constexpr uint32_t T_S = 0, T_P0 = 128, T_P1 = 192, T_O = 256;
+};
+
+struct SpTile {
+  int b, h, qb, n, start, bad;
+};
+
+struct SpCtrl {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full, s_free, p_full[2];
+  uint64_t o_full, o_ready;
+  uint64_t r_full, r_empty;
+  uint64_t ti_full[2], ti_empty[2];
+  uint64_t stg_ready, stg_full;
+  uint64_t drain;
+  SpTile ti[2];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+static_assert(sizeof(SpCtrl) <= 1024, "control block");
+
+template <typename CtrlT>
+__device__ __noinline__ bool sp_wait(uint64_t* bar, uint32_t parity, CtrlT& ctl, const AttnParams& p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 31u) == 0) {
+      if (ctl.abort_flag) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        ctl.abort_flag = 1;
+        record_status(p.status, RT_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void sp_decode(const AttnParams& p, int tile, int& b, int& h, int& qb) {
+  qb = tile % p.nqb;
+  const int rest = tile / p.nqb;
+  h = rest % p.H;
+  b = rest / p.H;
+}
+
+// ------------------------------------------------------------------ producer
+template <int DPAD>
+__device__ __forceinline__ void sp_producer(const TmaSet& tm, const AttnParams& p, SpCtrl& ctl, uint8_t* base,
+                                            int ntiles) {
+  using C = SpCfg<DPAD>;
+  const int lane = threadIdx.x & 31;
+  uint8_t* sQ = base + C::OFF_Q;
+  uint8_t* sStage = base + C::OFF_STAGE;
+  uint8_t* sR = base + C::OFF_R;
+  uint32_t g = 0, qi = 0, ri = 0;          // block, Q-load and R-load counters
+  int issued_q = 0, issued_r = 0;          // for the drain on abort
+  bool ok = true;
+  int it = 0;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+    const int slot = it & 1;
+    if (it >= 2) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.ti_empty[slot], ((it >> 1) - 1) & 1, ctl, p));
+      if (!ok) break;
+    }
+    int b, h, qb;
+    sp_decode(p, tile, b, h, qb);
+    const int row = (p.Hm == 1 ? 0 : h) * p.nqb + qb;
+    int start = 0, end = 0, bad = 0;
+    if (lane == 0) {
+      start = __ldg(p.row_ptr + row);
+      end = __ldg(p.row_ptr + row + 1);
+      if (start < 0 || end < start || static_cast<long long>(end) > p.nnz || end - start > p.nkb) bad = 1;
+    }
+    start = __shfl_sync(0xffffffffu, start, 0);
+    end = __shfl_sync(0xffffffffu, end, 0);
+    bad = __shfl_sync(0xffffffffu, bad, 0);
+    if (!bad) {
+      for (int i = lane; i < end - start; i += 32) {
+        const int c = __ldg(p.col_idx + start + i);
+        const int prev = i > 0 ? __ldg(p.col_idx + start + i - 1) : -1;
+        if (c < 0 || c >= p.nkb || c <= prev) bad = 1;
+      }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    const int n = bad ? 0 : end - start;
+    if (lane == 0) {
+      ctl.ti[slot] = SpTile{b, h, qb, n, start, bad};
+      if (bad) record_status(p.status, RT_ERR_BAD_INDEX);
+      mbar_arrive(&ctl.ti_full[slot]);
+    }
+    __syncwarp();
+    if (bad) continue;
+    if (lane == 0) {
+      const int q_row = qb * 128;
+      if (n > 0) {
+        const int qs = C::QBUF == 2 ? (qi & 1) : 0;
+        if (qi >= static_cast<uint32_t>(C::QBUF) &&
+            !sp_wait(&ctl.q_empty[qs], ((qi / C::QBUF) - 1) & 1, ctl, p)) ok = false;
+        if (ok) {
+          uint8_t* q = sQ + qs * C::TILE_BYTES;
+          mbar_arrive_expect_tx(&ctl.q_full[qs], C::TILE_BYTES);
+          tma_load_4d(q, &tm.q[0], &ctl.q_full[qs], 0, q_row, h, b);
+          if (C::C1) tma_load_4d(q + 128 * 128, &tm.q[1], &ctl.q_full[qs], 64, q_row, h, b);
+          ++qi;
+          issued_q = 1;
+        }
+        for (int j = 0; ok && j < n; ++j, ++g) {
+          const int st = g % C::NST;
+          if (g >= static_cast<uint32_t>(C::NST) &&
+              !sp_wait(&ctl.kv_empty[st], ((g / C::NST) - 1) & 1, ctl, p)) { ok = false; break; }
+          const int kb = __ldg(p.col_idx + start + j);
+          uint8_t* sK = sStage + st * C::STAGE_BYTES;
+          uint8_t* sV = sK + C::TILE_BYTES;
+          mbar_arrive_expect_tx(&ctl.k_full[st], C::TILE_BYTES);
+          tma_load_4d(sK, &tm.k[0], &ctl.k_full[st], 0, kb * 128, h, b);
+          if (C::C1) tma_load_4d(sK + 128 * 128, &tm.k[1], &ctl.k_full[st], 64, kb * 128, h, b);
+          mbar_arrive_expect_tx(&ctl.v_full[st], C::TILE_BYTES);
+          tma_load_4d(sV, &tm.v[0], &ctl.v_full[st], 0, kb * 128, h, b);
+          if (C::C1) tma_load_4d(sV + 128 * 128, &tm.v[1], &ctl.v_full[st], 64, kb * 128, h, b);
+        }
+      }
+      // residual tile (bf16) for this tile's epilogue, once the previous epilogue released it
+      if (ok && !p.r_f32) {
+        if (ri >= 1 && !sp_wait(&ctl.r_empty, (ri - 1) & 1, ctl, p)) ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&ctl.r_full, C::TILE_BYTES);
+          tma_load_4d(sR, &tm.r[0], &ctl.r_full, 0, q_row, h, b);
+          if (C::C1) tma_load_4d(sR + 128 * 128, &tm.r[1], &ctl.r_full, 64, q_row, h, b);
+          ++ri;
+          issued_r = 1;
+        }
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  }
+  if (!ok && lane == 0) {
+    // let every copy this thread started land before shared memory is released
+    const uint64_t lim = p.wait_limit_ns;
+    if (issued_q)
+      for (uint32_t i = (qi > static_cast<uint32_t>(C::QBUF) ? qi - C::QBUF : 0); i < qi; ++i)
+        drain_wait(&ctl.q_full[C::QBUF == 2 ? (i & 1) : 0], (i / C::QBUF) & 1, lim);
+    if (issued_r) drain_wait(&ctl.r_full, (ri - 1) & 1, lim);
+    for (uint32_t i = (g > static_cast<uint32_t>(C::NST) ? g - C::NST : 0); i < g; ++i) {
+      drain_wait(&ctl.k_full[i % C::NST], (i / C::NST) & 1, lim);
+      drain_wait(&ctl.v_full[i % C::NST], (i / C::NST) & 1, lim);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int DPAD>
+__device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t* base, uint32_t tmem, int ntiles) {
+  using C = SpCfg<DPAD>;
+  constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t IDESC_PV_FULL = make_idesc_bf16(128, DPAD == 128 ? 128 : 64, 0, 1);
+  constexpr uint32_t IDESC_PV_C1 = make_idesc_bf16(128, C::C1 > 0 ? C::C1 : 16, 0, 1);
+  const uint32_t q0 = smem_u32(base + C::OFF_Q);
+  const uint32_t stage0 = smem_u32(base + C::OFF_STAGE);
+  uint32_t g = 0, qi = 0;
+  bool ok = true;
+
+  auto issue_pv = [&](uint32_t gi, bool first) -> bool {
+    const int st = gi % C::NST;
+    if (!sp_wait(&ctl.p_full[gi & 1], (gi >> 1) & 1, ctl, p)) return false;
+    if (!sp_wait(&ctl.v_full[st], (gi / C::NST) & 1, ctl, p)) return false;
+    tc_fence_after();
+    const uint32_t v_tile = stage0 + st * C::STAGE_BYTES + C::TILE_BYTES;
+    const uint32_t tp = tmem + ((gi & 1) ? C::T_P1 : C::T_P0);
+    const uint32_t dst = tmem + C::T_O;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+      mma_ts(dst, tp + kk * 8, v_desc_c0<DPAD, 128>(v_tile, kk), IDESC_PV_FULL, acc);
+      if (C::C1 > 0 && DPAD != 128)
+        mma_ts(dst + 64, tp + kk * 8, v_desc_c1<DPAD, 128>(v_tile, kk), IDESC_PV_C1, acc);
+    }
+    mma_commit(&ctl.kv_empty[st]);
+    mma_commit(&ctl.o_ready);
+    return true;
+  };
+
+  int it = 0;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+    const int slot = it & 1;
+    if (!sp_wait(&ctl.ti_full[slot], (it >> 1) & 1, ctl, p)) { ok = false; break; }
+    const int n = ctl.ti[slot].n;
+    if (n > 0) {
+      const int qs = C::QBUF == 2 ? (qi & 1) : 0;
+      if (!sp_wait(&ctl.q_full[qs], (qi / C::QBUF) & 1, ctl, p)) { ok = false; break; }
+      const uint32_t q_addr = q0 + qs * C::TILE_BYTES;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int st = g % C::NST;
+        if (!sp_wait(&ctl.k_full[st], (g / C::NST) & 1, ctl, p)) { ok = false; break; }
+        if (g > 0 && !sp_wait(&ctl.s_free, (g - 1) & 1, ctl, p)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t k_tile = stage0 + st * C::STAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < DPAD / 16; ++kk)
+          mma_ss(tmem + C::T_S, kmajor_desc<DPAD>(q_addr, 128, kk), kmajor_desc<DPAD>(k_tile, 128, kk),
+                 IDESC_QK, kk > 0 ? 1u : 0u);
+        mma_commit(&ctl.s_full);
+        if (j == n - 1) mma_commit(&ctl.q_empty[qs]);
+        if (j > 0 && !issue_pv(g - 1, j == 1)) { ok = false; break; }
+      }
+      if (!ok) break;
+      if (!issue_pv(g - 1, n == 1)) { ok = false; break; }
+      mma_commit(&ctl.o_full);
+      ++qi;
+    }
+    mbar_arrive(&ctl.ti_empty[slot]);
+  }
+  if (!ok) {
+    mma_commit(&ctl.drain);
+    drain_wait(&ctl.drain, 0, p.wait_limit_ns);
+  }
+}
+
+// ------------------------------------------------------------------ softmax + epilogue
+template <int DPAD>
+__device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p, SpCtrl& ctl, uint8_t* base,
+                                           uint32_t tmem, int ntiles) {
+  using C = SpCfg<DPAD>;
+  const int t = threadIdx.x;
+  const int warp = t >> 5;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tS = tmem + lane_base + C::T_S;
+  const uint32_t tO = tmem + lane_base + C::T_O;
+  uint8_t* sR = base + C::OFF_R;
+  uint8_t* sOst = base + C::OFF_OST;
+  const float sl2 = p.scale_log2;
+  uint32_t g = 0, oi = 0, ri = 0, si = 0;
+  bool ok = true;
+  int it = 0;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+    const int slot = it & 1;
+    ok = __all_sync(0xffffffffu, sp_wait(&ctl.ti_full[slot], (it >> 1) & 1, ctl, p));
+    if (!ok) break;
+    const SpTile ti = ctl.ti[slot];
+    mbar_arrive(&ctl.ti_empty[slot]);
+    if (ti.bad) continue;
+    const int grow = ti.qb * 128 + t;
+    const size_t rho_idx = (static_cast<size_t>(ti.b) * p.H + ti.h) * p.L + grow;
+    const float rho = grow < p.L ? __ldg(p.rho_in + rho_idx) : 0.f;
+    float m = 0.f, l = 0.f;
+    for (int j = 0; j < ti.n; ++j, ++g) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full, g & 1, ctl, p));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      load_scores<128>(tS, s);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&ctl.s_free);
+      const int kb = __ldg(p.col_idx + ti.start + j);
+      mask_tail<128>(s, p.L - kb * 128);
+      const float mx = row_max<128>(s) * sl2;
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+        const float m_new = fmaxf(m, mx);
+        const float alpha = ex2_approx(m - m_new);
+        l *= alpha;
+        ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_ready, (g - 1) & 1, ctl, p));
+        if (!ok) break;
+        tc_fence_after();
+        rescale_row<DPAD>(tO, alpha);
+        m = m_new;
+      }
+      const uint32_t tP = tmem + lane_base + ((g & 1) ? C::T_P1 : C::T_P0);
+      l += exp_pack_store<128>(s, sl2, m, tP);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ctl.p_full[g & 1]);
+    }
+    if (!ok) break;
+    // ------------------------------------------------------------- epilogue
+    if (ti.n > 0) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_full, oi & 1, ctl, p));
+      if (!ok) break;
+      tc_fence_after();
+      ++oi;
+    }
+    if (!p.r_f32) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.r_full, ri & 1, ctl, p));
+      if (!ok) break;
+    }
+    const float rho_hat = fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add));
+    const float scale = ti.n > 0 ? rho_hat / l : 0.f;
+    uint32_t packed[DPAD / 2];
+#pragma unroll
+    for (int c = 0; c < DPAD; c += 16) {
+      uint32_t acc[16];
+      if (ti.n > 0) { tmem_ld_x16(tO + c, acc); tmem_wait_ld(); }
+      float rr[16];
+      if (p.r_f32) {
+        if (grow < p.L) {
+          const float4* src = reinterpret_cast<const float4*>(
+              static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
+              static_cast<long long>(grow) * p.stride_l + c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v4 = (c + 4 * u < p.d) ? __ldg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            rr[4 * u] = v4.x; rr[4 * u + 1] = v4.y; rr[4 * u + 2] = v4.z; rr[4 * u + 3] = v4.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+        }
+      } else {
+        load_row16<DPAD>(sR, 128, t, c, false, rr);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a0 = (ti.n > 0 ? __uint_as_float(acc[2 * i]) * scale : 0.f) + rr[2 * i];
+        const float a1 = (ti.n > 0 ? __uint_as_float(acc[2 * i + 1]) * scale : 0.f) + rr[2 * i + 1];
+        packed[c / 2 + i] = pack_bf16x2(a0, a1);
+      }
+    }
+    if (!p.r_f32) {
+      mbar_arrive(&ctl.r_empty);
+      ++ri;
+    }
+    // staging slot: thread 0 makes sure the store that last used it has read it
+    const int ss = C::OSTG == 2 ? (si & 1) : 0;
+    if (t == 0) {
+      if (C::OSTG == 2) tma_store_wait_read<1>(); else tma_store_wait_read<0>();
+      mbar_arrive(&ctl.stg_ready);
+    }
+    ok = __all_sync(0xffffffffu, sp_wait(&ctl.stg_ready, si & 1, ctl, p));
+    if (!ok) break;
+    uint8_t* ost = sOst + ss * C::TILE_BYTES;
+#pragma unroll
+    for (int c = 0; c < DPAD; c += 16) {
+      const bool c1 = c >= 64;
+      const uint32_t rb = c1 ? C::C1B : 128;
+      const uint32_t cbase = c1 ? 128 * 128 : 0;
+      const int col = c1 ? c - 64 : c;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        uint4 w;
+        w.x = packed[c / 2 + 4 * u + 0];
+        w.y = packed[c / 2 + 4 * u + 1];
+        w.z = packed[c / 2 + 4 * u + 2];
+        w.w = packed[c / 2 + 4 * u + 3];
+        *reinterpret_cast<uint4*>(ost + cbase + swz_off(t * rb + (col * 2 + u * 16), rb)) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&ctl.stg_full);
+    if (t == 0) {
+      if (sp_wait(&ctl.stg_full, si & 1, ctl, p)) {
+        const int q_row = ti.qb * 128;
+        tma_store_4d(&tm.o[0], ost, 0, q_row, ti.h, ti.b);
+        if (C::C1) tma_store_4d(&tm.o[1], ost + 128 * 128, 64, q_row, ti.h, ti.b);
+        tma_store_commit();
+      }
+    }
+    __syncwarp();
+    ++si;
+  }
+  if (t == 0) tma_store_wait0();
+}
+
+template <int DPAD>
+__global__ void __launch_bounds__(kThreads, 1)
+sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles) {
+  using C = SpCfg<DPAD>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  SpCtrl& ctl = *reinterpret_cast<SpCtrl*>(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl.q_full[i], 1);
+      mbar_init(&ctl.q_empty[i], 1);
+      mbar_init(&ctl.p_full[i], kSoftmaxThreads);
+      mbar_init(&ctl.ti_full[i], 1);
+      mbar_init(&ctl.ti_empty[i], kSoftmaxThreads + 1);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&ctl.k_full[i], 1);
+      mbar_init(&ctl.v_full[i], 1);
+      mbar_init(&ctl.kv_empty[i], 1);
+    }
+    mbar_init(&ctl.s_full, 1);
+    mbar_init(&ctl.s_free, kSoftmaxThreads);
+    mbar_init(&ctl.o_full, 1);
+    mbar_init(&ctl.o_ready, 1);
+    mbar_init(&ctl.r_full, 1);
+    mbar_init(&ctl.r_empty, kSoftmaxThreads);
+    mbar_init(&ctl.stg_ready, 1);
+    mbar_init(&ctl.stg_full, kSoftmaxThreads);
+    mbar_init(&ctl.drain, 1);
+    ctl.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&ctl.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == kProducerWarp) {
+    sp_producer<DPAD>(tm, p, ctl, base, ntiles);
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) sp_mma<DPAD>(p, ctl, base, tmem, ntiles);
+  } else {
+    sp_softmax<DPAD>(tm, p, ctl, base, tmem, ntiles);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace rtb

@@ -285,6 +285,27 @@ def test_bad_row_ptr_recorded():
     assert _bad_index_run([0, 3, 2], [0, 1], 2) == rt.RT_ERR_BAD_INDEX
 
 
+def test_sparse_step_bad_row_recorded_good_rows_correct():
+    """One corrupt CSR row among good ones: the persistent sparse kernel records
+    RT_ERR_BAD_INDEX, skips that tile and still computes every other tile."""
+    B, H, L, d, blk = 1, 2, 512, 64, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=51, device=DEV)
+    mask = np.array([[[1, 0, 0, 0], [1, 1, 0, 0], [0, 1, 1, 0], [0, 0, 1, 1]]], dtype=np.uint8)
+    rp, ci = ref.build_block_index_ref(mask)
+    ci_bad = ci.copy()
+    ci_bad[rp[2]] = 9                                         # row 2 points past nkb
+    idx = rt.make_block_index(torch.from_numpy(rp).to(DEV), torch.from_numpy(ci_bad).to(DEV), 1, 4, 4)
+    rho_s, r_s = _stats_inputs((B, H, L, d), 52)
+    o = torch.zeros_like(q)
+    rt.rt_sparse_step(q, k, v, idx, rho_s, r_s, block=blk, lam=0.04, step_distance=2, o=o)
+    assert rt.rt_check_device_error() == rt.RT_ERR_BAD_INDEX
+    want = ref.sparse_step_ref(f64(q), f64(k), f64(v), mask, blk, f64(rho_s), f64(r_s), 0.04, 2)
+    got = f64(o)
+    good = np.r_[0:256, 384:512]
+    check_out(got[:, :, good], want[:, :, good], "good rows")
+    assert np.all(got[:, :, 256:384] == 0)                   # the bad tile wrote nothing
+
+
 def test_good_index_after_errors_still_correct():
     test_workload_cycle_full("tiny")
 
