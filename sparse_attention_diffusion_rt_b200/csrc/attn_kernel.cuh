@@ -117,7 +117,7 @@ __device__ __forceinline__ void record_status(unsigned int* status, unsigned int
 
 // Bounded mbarrier wait.  Returns false after a timeout (recorded) or when
 // another role of the CTA has already aborted.
-static __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctrl& ctl,
+static __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctrl& ctl,
                                       const AttnParams& p) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();

@@ -73,7 +73,7 @@ struct SpCtrl {
 static_assert(sizeof(SpCtrl) <= 1024, "control block");
 
 template <typename CtrlT>
-__device__ __noinline__ bool sp_wait(uint64_t* bar, uint32_t parity, CtrlT& ctl, const AttnParams& p) {
+__device__ __forceinline__ bool sp_wait(uint64_t* bar, uint32_t parity, CtrlT& ctl, const AttnParams& p) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
