@@ -16,12 +16,11 @@ __device__ __forceinline__ float row_max(const uint32_t (&s)[BN]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
 #pragma unroll
-  for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
-#pragma unroll
-  for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-  return mx[0];
+  for (int c = 8; c < BN; c += 2)
+    mx[(c >> 1) & 7] = max3f(mx[(c >> 1) & 7], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+  const float a = max3f(mx[0], mx[1], mx[2]);
+  const float b = max3f(mx[3], mx[4], mx[5]);
+  return max3f(a, b, fmaxf(mx[6], mx[7]));
 }
 
 // Set logits of key columns >= valid (keys past the end of the sequence) to -inf.
@@ -39,28 +38,31 @@ __device__ __forceinline__ void mask_tail(uint32_t (&s)[BN], int valid) {
 // (of the fp32 values).  The caller waits for the stores (tmem_wait_st).
 template <int BN>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BN], float sl2, float m, uint32_t tP) {
-  float sum[8];
+  uint64_t sum[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sum[i] = 0.f;
-  const float neg_m = -m;
+  for (int i = 0; i < 4; ++i) sum[i] = 0ull;
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t neg_m2 = f2_pack(-m, -m);
 #pragma unroll
   for (int c0 = 0; c0 < BN; c0 += 64) {
     uint32_t pk[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-      const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c]), sl2, neg_m));
-      const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * c + 1]), sl2, neg_m));
-      sum[(2 * c) & 7] += p0;
-      sum[(2 * c + 1) & 7] += p1;
+      const uint64_t x = ffma2(f2_pack(__uint_as_float(s[c0 + 2 * c]), __uint_as_float(s[c0 + 2 * c + 1])),
+                               scale2, neg_m2);
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      const float p0 = ex2_approx(x0);
+      const float p1 = ex2_approx(x1);
+      sum[c & 3] = fadd2(sum[c & 3], f2_pack(p0, p1));
       pk[c] = pack_bf16x2(p0, p1);
     }
     tmem_st_x32(tP + c0 / 2, pk);
   }
-#pragma unroll
-  for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) sum[i] += sum[i + w];
-  return sum[0];
+  const uint64_t t = fadd2(fadd2(sum[0], sum[1]), fadd2(sum[2], sum[3]));
+  float lo, hi;
+  f2_unpack(t, lo, hi);
+  return lo + hi;
 }
 
 // Load BN fp32 logits of this thread's row from TMEM (caller waits with tmem_wait_ld).
