@@ -7,6 +7,7 @@
 
 #include "attn_kernel.cuh"
 #include "sparse_kernel.cuh"
+#include "pp_sparse.cuh"
 
 namespace rtb {
 
@@ -76,6 +77,29 @@ cudaError_t launch_sparse_impl(const TmaSet& tm, const AttnParams& p, cudaStream
   const long long ntiles = static_cast<long long>(p.B) * p.H * p.nqb;
   const int grid = static_cast<int>(ntiles < sm_count[dev & 63] ? ntiles : sm_count[dev & 63]);
   kern<<<grid, kThreads, smem, s>>>(tm, p, static_cast<int>(ntiles));
+  return cudaGetLastError();
+}
+
+// Ping-pong persistent sparse-step kernel (d <= 64, 128-token blocks).
+template <int DPAD>
+cudaError_t launch_pp_sparse(const TmaSet& tm, const AttnParams& p, cudaStream_t s) {
+  static std::atomic<unsigned long long> configured{0};
+  static int sm_count[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(pp_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, PpCfg::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sm_count[dev & 63], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const long long ntiles = static_cast<long long>(p.B) * p.H * p.nqb;
+  const long long half = (ntiles + 1) / 2;
+  const int grid = static_cast<int>(half < sm_count[dev & 63] ? half : sm_count[dev & 63]);
+  pp_sparse_kernel<64><<<grid, kPpThreads, PpCfg::SMEM, s>>>(tm, p, static_cast<int>(ntiles));
   return cudaGetLastError();
 }
 

@@ -55,6 +55,7 @@ struct SpCfg {
 
 struct SpTile {
   int b, h, qb, n, start, bad;
+  int tail_j, tail_valid;   // block index (in this row) that holds the sequence end, keys of it inside
 };
 
 struct SpCtrl {
@@ -138,7 +139,7 @@ __device__ __forceinline__ void sp_producer(const TmaSet& tm, const AttnParams& 
     bad = __any_sync(0xffffffffu, bad);
     const int n = bad ? 0 : end - start;
     if (lane == 0) {
-      ctl.ti[slot] = SpTile{b, h, qb, n, start, bad};
+      ctl.ti[slot] = SpTile{b, h, qb, n, start, bad, -1, 128};
       if (bad) record_status(p.status, RT_ERR_BAD_INDEX);
       mbar_arrive(&ctl.ti_full[slot]);
     }
