@@ -147,6 +147,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+// Calibration visits every key block in ascending order; the CTAs of a head
+// then stream the same K/V blocks at about the same time and share them in L2
+// (a per-CTA rotated order measured slower).
+__device__ __forceinline__ int cal_kb(const AttnParams&, int, int j) { return j; }
+
 __device__ __forceinline__ bool is_kept(const Ctrl& ctl, int kb) {
   return (ctl.kept_bits[kb >> 5] >> (kb & 31)) & 1u;
 }
@@ -207,7 +212,7 @@ __device__ __forceinline__ void producer_role(const TmaSet& tm, const AttnParams
     const int st = j % C::NST;
     const uint32_t use = j / C::NST;
     if (j >= C::NST && !wait_bar(&ctl.kv_empty[st], (use - 1) & 1, ctl, p)) { ok = false; break; }
-    const int kb = CAL ? j : __ldg(p.col_idx + ctl.row_start + j);
+    const int kb = CAL ? cal_kb(p, qb, j) : __ldg(p.col_idx + ctl.row_start + j);
     uint8_t* sK = sStage + st * C::STAGE_BYTES;
     uint8_t* sV = sK + C::KT_BYTES;
     mbar_arrive_expect_tx(&ctl.k_full[st], C::KT_BYTES);
@@ -256,7 +261,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Ctrl& ctl, uint8_t
     uint32_t dst = tmem + C::T_O;
     bool first = (i == 0);
     if (CAL) {
-      const bool kept = is_kept(ctl, i);
+      const bool kept = is_kept(ctl, cal_kb(p, blockIdx.x, i));
       dst = tmem + (kept ? C::T_O : C::T_OUT);
       first = kept ? first_in : first_out;
       if (kept) first_in = false; else first_out = false;
@@ -386,7 +391,7 @@ __device__ __forceinline__ void softmax_role(const TmaSet& tm, const AttnParams&
     tc_fence_before();
     mbar_arrive(&ctl.s_free);
 
-    const int kb = CAL ? j : __ldg(p.col_idx + ctl.row_start + j);
+    const int kb = CAL ? cal_kb(p, qb, j) : __ldg(p.col_idx + ctl.row_start + j);
     mask_tail<BN>(s, p.L - kb * BN);                 // keys past the end of the sequence
     const float mx = row_max<BN>(s) * sl2;
     if (j == 0) {

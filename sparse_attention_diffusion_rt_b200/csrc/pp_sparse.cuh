@@ -8,10 +8,9 @@
 // barrier latency and tensor-core work.  CTA c handles tiles c + i*gridDim.x;
 // even i go to pipeline A, odd i to B.
 //
-// Threads (320): warps 0-3 softmax + epilogue of A, warps 4-7 of B (thread t
+// Threads (352): warps 0-3 softmax + epilogue of A, warps 4-7 of B (thread t
 // owns TMEM lane t % 128), lanes 0 and 1 of warp 8 are the TMA producers of A
-// and B, lane 0 of warp 9 issues the MMAs of both pipelines from a
-// non-blocking scheduler.
+// and B, lane 0 of warps 9 and 10 issue the MMAs of A and B.
 // TMEM: pipeline p uses columns [256p, 256p+256): S logits [0,128), bf16 P
 // [128,192), O [192,256).  A pipeline's next QK^T is issued as soon as its
 // softmax has read the current logits (s_free), so it runs under that softmax;
@@ -31,9 +30,9 @@
 
 namespace rtb {
 
-constexpr int kPpThreads = 320;
+constexpr int kPpThreads = 352;
 constexpr int kPpProducerWarp = 8;
-constexpr int kPpMmaWarp = 9;
+constexpr int kPpMmaWarp = 9;        // warps 9 and 10: MMA issuers of pipelines A and B
 
 struct PpCfg {
   static constexpr int TILE = 128 * 64 * 2;                 // bf16 [128][64]
@@ -57,7 +56,7 @@ struct PpPipe {
 
 struct PpCtrl {
   PpPipe pipe[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -148,118 +147,76 @@ __device__ __forceinline__ void pp_producer(const TmaSet& tm, const AttnParams& 
   }
 }
 
-// ------------------------------------------------------------------ MMA scheduler (both pipelines)
-// Per pipeline the scheduler keeps two cursors over the blocks of the current
-// tile: the next QK^T (needs its K tile, the tile's Q for the first block, and
-// the softmax to have read the previous logits) and the next PV (needs P and
-// the V tile).  Every readiness test is non-blocking so that one pipeline never
-// holds back the other.
-struct PpMmaState {
-  int it, n, jq, jp, have_tile;  // tile iteration, blocks in tile, next QK, next PV, tile info read
-  uint32_t gq, gp, qi;           // global block counters of the next QK / PV, Q loads consumed
-  bool done;
-};
-
-__device__ __forceinline__ bool pp_mma_step(PpMmaState& S, int pipe, PpCtrl& ctl, uint32_t tmem, uint8_t* pbase,
-                                            int ntiles) {
+// ------------------------------------------------------------------ MMA issuer (one thread per pipeline)
+// Lane 0 of warp 9 + pipe issues pipeline `pipe`'s MMAs: QK^T of block j+1 as
+// soon as the softmax has read block j's logits (s_free), then PV of block j
+// once P is written (p_full).  tcgen05.commit tracks the issuing thread's own
+// MMAs, so each pipeline's barriers see only its own work.
+__device__ __forceinline__ void pp_mma(const AttnParams& p, PpCtrl& ctl, uint8_t* pbase, uint32_t tmem, int pipe,
+                                       int ntiles) {
   using C = PpCfg;
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t IDESC_PV = make_idesc_bf16(128, 64, 0, 1);
-  if (S.done) return false;
   PpPipe& P = ctl.pipe[pipe];
   const uint32_t tbase = tmem + 256u * pipe;
-  if (!S.have_tile) {
-    if (pp_tile(S.it, pipe) >= ntiles) { S.done = true; return true; }
-    const int slot = S.it & 1;
-    if (!mbar_test_wait(&P.ti_full[slot], (S.it >> 1) & 1)) return false;
-    const int n = P.ti[slot].n;
-    if (n == 0) {
-      mbar_arrive(&P.ti_empty[slot]);
-      ++S.it;
-      return true;
-    }
-    S.n = n;
-    S.jq = 0;
-    S.jp = 0;
-    S.have_tile = 1;
-    return true;
-  }
-  bool prog = false;
-  if (S.jq < S.n) {
-    const int st = S.gq & 1;
-    const bool ready = (S.jq > 0 || mbar_test_wait(&P.q_full, S.qi & 1)) &&
-                       mbar_test_wait(&P.k_full[st], (S.gq >> 1) & 1) &&
-                       (S.gq == 0 || mbar_test_wait(&P.s_free, (S.gq - 1) & 1));
-    if (ready) {
-      tc_fence_after();
-      const uint32_t q_addr = smem_u32(pbase + C::Q);
-      const uint32_t k_tile = smem_u32(pbase + C::STAGE + st * 2 * C::TILE);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tbase, kmajor_desc<64>(q_addr, 128, kk), kmajor_desc<64>(k_tile, 128, kk), IDESC_QK,
-               kk > 0 ? 1u : 0u);
-      mma_commit(&P.s_full);
-      if (S.jq == S.n - 1) mma_commit(&P.q_empty);
-      ++S.jq;
-      ++S.gq;
-      prog = true;
-    }
-  }
-  if (S.jp < S.jq) {
-    const int st = S.gp & 1;
-    if (mbar_test_wait(&P.p_full, S.gp & 1) && mbar_test_wait(&P.v_full[st], (S.gp >> 1) & 1)) {
-      tc_fence_after();
-      const uint32_t v_tile = smem_u32(pbase + C::STAGE + st * 2 * C::TILE + C::TILE);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(tbase + 192, tbase + 128 + kk * 8, v_desc_c0<64, 128>(v_tile, kk), IDESC_PV,
-               (S.jp == 0 && kk == 0) ? 0u : 1u);
-      mma_commit(&P.kv_empty[st]);
-      mma_commit(&P.pv_done);
-      ++S.gp;
-      if (++S.jp == S.n) {
-        mma_commit(&P.o_full);
-        mbar_arrive(&P.ti_empty[S.it & 1]);
-        ++S.qi;
-        ++S.it;
-        S.have_tile = 0;
-      }
-      prog = true;
-    }
-  }
-  return prog;
-}
-
-static_assert(kPpMmaWarp == kPpThreads / 32 - 1, "MMA warp is the last warp");
-
-__device__ __forceinline__ void pp_mma(const AttnParams& p, PpCtrl& ctl, uint8_t* smem_pipes, uint32_t tmem,
-                                       int ntiles) {
-  PpMmaState st[2] = {{0, 0, 0, 0, 0, 0u, 0u, 0u, false}, {0, 0, 0, 0, 0, 0u, 0u, 0u, false}};
-  uint64_t last = globaltimer_ns();
-  uint32_t idle = 0;
+  const uint32_t q_addr = smem_u32(pbase + C::Q);
+  const uint32_t stage0 = smem_u32(pbase + C::STAGE);
+  uint32_t g = 0, qi = 0;
   bool ok = true;
-  while (!(st[0].done && st[1].done)) {
-    bool prog = pp_mma_step(st[0], 0, ctl, tmem, smem_pipes, ntiles);
-    prog |= pp_mma_step(st[1], 1, ctl, tmem, smem_pipes + PpCfg::PIPE_BYTES, ntiles);
-    if (prog) {
-      idle = 0;
-      continue;
-    }
-    if ((++idle & 63u) == 0) {
-      const uint64_t now = globaltimer_ns();
-      if (idle == 64) last = now;
-      if (ctl.abort_flag) { ok = false; break; }
-      if (now - last > p.wait_limit_ns) {
-        ctl.abort_flag = 1;
-        record_status(p.status, RT_ERR_TIMEOUT);
-        ok = false;
-        break;
+
+  auto issue_qk = [&](uint32_t gq, bool first_of_tile) -> bool {
+    const int st = gq & 1;
+    if (first_of_tile && !pp_wait(&P.q_full, qi & 1, ctl, p)) return false;
+    if (!pp_wait(&P.k_full[st], (gq >> 1) & 1, ctl, p)) return false;
+    if (gq > 0 && !pp_wait(&P.s_free, (gq - 1) & 1, ctl, p)) return false;
+    tc_fence_after();
+    const uint32_t k_tile = stage0 + st * 2 * C::TILE;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(tbase, kmajor_desc<64>(q_addr, 128, kk), kmajor_desc<64>(k_tile, 128, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+    mma_commit(&P.s_full);
+    return true;
+  };
+  auto issue_pv = [&](uint32_t gp, bool first_of_tile) -> bool {
+    const int st = gp & 1;
+    if (!pp_wait(&P.p_full, gp & 1, ctl, p)) return false;
+    if (!pp_wait(&P.v_full[st], (gp >> 1) & 1, ctl, p)) return false;
+    tc_fence_after();
+    const uint32_t v_tile = stage0 + st * 2 * C::TILE + C::TILE;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(tbase + 192, tbase + 128 + kk * 8, v_desc_c0<64, 128>(v_tile, kk), IDESC_PV,
+             (first_of_tile && kk == 0) ? 0u : 1u);
+    mma_commit(&P.kv_empty[st]);
+    mma_commit(&P.pv_done);
+    return true;
+  };
+
+  for (int it = 0; ok; ++it) {
+    if (pp_tile(it, pipe) >= ntiles) break;
+    const int slot = it & 1;
+    if (!pp_wait(&P.ti_full[slot], (it >> 1) & 1, ctl, p)) { ok = false; break; }
+    const int n = P.ti[slot].n;
+    if (n > 0) {
+      if (!issue_qk(g, true)) { ok = false; break; }
+      if (n == 1) mma_commit(&P.q_empty);
+      for (int j = 0; j < n; ++j) {
+        if (j + 1 < n) {
+          if (!issue_qk(g + 1, false)) { ok = false; break; }
+          if (j + 2 == n) mma_commit(&P.q_empty);
+        }
+        if (!issue_pv(g, j == 0)) { ok = false; break; }
+        ++g;
       }
+      if (!ok) break;
+      mma_commit(&P.o_full);
+      ++qi;
     }
+    mbar_arrive(&P.ti_empty[slot]);
   }
   if (!ok) {
-    mma_commit(&ctl.drain);
-    drain_wait(&ctl.drain, 0, p.wait_limit_ns);
+    mma_commit(&ctl.drain[pipe]);
+    drain_wait(&ctl.drain[pipe], 0, p.wait_limit_ns);
   }
 }
 
@@ -349,31 +306,37 @@ __device__ __forceinline__ void pp_softmax(const TmaSet& tm, const AttnParams& p
     ok = __all_sync(0xffffffffu, pp_wait(&P.stg_ready, si & 1, ctl, p));
     if (!ok) break;
 #pragma unroll
-    for (int c = 0; c < 64; c += 16) {
-      uint32_t acc[16];
-      if (ti.n > 0) { tmem_ld_x16(tO + c, acc); tmem_wait_ld(); }
-      float rr[16];
-      if (p.r_f32) {
-        if (grow < p.L) {
-          const float4* src = reinterpret_cast<const float4*>(
-              static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
-              static_cast<long long>(grow) * p.stride_l + c);
+    for (int h0 = 0; h0 < 64; h0 += 32) {
+      uint32_t acc[32];
+      if (ti.n > 0) {
+        tmem_ld_x32(tO + h0, acc);
+        tmem_wait_ld();
+      }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4 v4 = (c + 4 * u < p.d) ? __ldg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-            rr[4 * u] = v4.x; rr[4 * u + 1] = v4.y; rr[4 * u + 2] = v4.z; rr[4 * u + 3] = v4.w;
+      for (int c = h0; c < h0 + 32; c += 16) {
+        float rr[16];
+        if (p.r_f32) {
+          if (grow < p.L) {
+            const float4* src = reinterpret_cast<const float4*>(
+                static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
+                static_cast<long long>(grow) * p.stride_l + c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 v4 = (c + 4 * u < p.d) ? __ldg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+              rr[4 * u] = v4.x; rr[4 * u + 1] = v4.y; rr[4 * u + 2] = v4.z; rr[4 * u + 3] = v4.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) rr[i] = 0.f;
           }
         } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+          load_row16<64>(sR, 128, t, c, false, rr);
         }
-      } else {
-        load_row16<64>(sR, 128, t, c, false, rr);
-      }
-      float o16[16];
+        float o16[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o16[i] = (ti.n > 0 ? __uint_as_float(acc[i]) * scale : 0.f) + rr[i];
-      store_row16<64>(sOst, 128, t, c, false, o16);
+        for (int i = 0; i < 16; ++i) o16[i] = (ti.n > 0 ? __uint_as_float(acc[c - h0 + i]) * scale : 0.f) + rr[i];
+        store_row16<64>(sOst, 128, t, c, false, o16);
+      }
     }
     if (!p.r_f32) {
       mbar_arrive(&P.r_empty);
@@ -426,7 +389,8 @@ pp_sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntil
       mbar_init(&P.stg_ready, 1);
       mbar_init(&P.stg_full, kSoftmaxThreads);
     }
-    mbar_init(&ctl.drain, 1);
+    mbar_init(&ctl.drain[0], 1);
+    mbar_init(&ctl.drain[1], 1);
     ctl.abort_flag = 0;
     fence_mbar_init();
   }
@@ -445,7 +409,8 @@ pp_sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntil
   } else if (warp == kPpProducerWarp) {
     if (lane < 2) pp_producer(tm, p, ctl, pipes + lane * C::PIPE_BYTES, lane, ntiles);
   } else if (lane == 0) {
-    pp_mma(p, ctl, pipes, tmem, ntiles);
+    const int pipe = warp - kPpMmaWarp;
+    pp_mma(p, ctl, pipes + pipe * C::PIPE_BYTES, tmem, pipe, ntiles);
   }
   tc_fence_before();
   __syncthreads();

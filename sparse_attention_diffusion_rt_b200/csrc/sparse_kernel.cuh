@@ -6,8 +6,7 @@
 // plus the cached residual of the masked tokens; reply to Pwod's W1: ramp-up).
 //
 // One CTA per SM walks the (batch, head, query block) tiles tile = blockIdx.x
-// + i * gridDim.x, query block fastest so that concurrent CTAs share the
-// head's K/V in L2.  Roles (192 threads):
+// + i * gridDim.x, (batch, head) fastest (see sp_decode).  Roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
 //   warp 4     producer: validates each tile's CSR row (all lanes), then lane 0
 //              issues the TMA loads: Q (double-buffered for d <= 96), the kept
@@ -91,11 +90,15 @@ __device__ __forceinline__ bool sp_wait(uint64_t* bar, uint32_t parity, CtrlT& c
   }
 }
 
+// Tile order: (batch, head) fastest, then query block.  Concurrent CTAs then
+// spread over many heads, so key blocks that every query block keeps (text
+// tokens) are not fetched by every SM at once, while each head's local key
+// blocks are still shared in L2 by the few neighbouring query blocks in flight.
 __device__ __forceinline__ void sp_decode(const AttnParams& p, int tile, int& b, int& h, int& qb) {
-  qb = tile % p.nqb;
-  const int rest = tile / p.nqb;
-  h = rest % p.H;
-  b = rest / p.H;
+  const int bh = tile % (p.B * p.H);
+  qb = tile / (p.B * p.H);
+  b = bh / p.H;
+  h = bh % p.H;
 }
 
 // ------------------------------------------------------------------ producer
