@@ -8,7 +8,7 @@ cudaError_t launch_attn_d64(bool cal, int block, const TmaSet& tm, const AttnPar
   if (block == 64) return cal ? launch_attn_impl<64, 64, true>(tm, p, grid, s)
                             : launch_attn_impl<64, 64, false>(tm, p, grid, s);
   if (block != 128) return cudaErrorInvalidValue;
-  return cal ? launch_attn_impl<64, 128, true>(tm, p, grid, s) : launch_pp_sparse<64>(tm, p, s);
+  return cal ? launch_pp_calibrate<64>(tm, p, s) : launch_pp_sparse<64>(tm, p, s);
 }
 
 }  // namespace rtb

@@ -8,6 +8,7 @@
 #include "attn_kernel.cuh"
 #include "sparse_kernel.cuh"
 #include "pp_sparse.cuh"
+#include "pp_calibrate.cuh"
 
 namespace rtb {
 
@@ -100,6 +101,24 @@ cudaError_t launch_pp_sparse(const TmaSet& tm, const AttnParams& p, cudaStream_t
   const long long half = (ntiles + 1) / 2;
   const int grid = static_cast<int>(half < sm_count[dev & 63] ? half : sm_count[dev & 63]);
   pp_sparse_kernel<64><<<grid, kPpThreads, PpCfg::SMEM, s>>>(tm, p, static_cast<int>(ntiles));
+  return cudaGetLastError();
+}
+
+// Ping-pong calibration kernel (d <= 64, 128-token blocks): two query tiles per CTA.
+template <int DPAD>
+cudaError_t launch_pp_calibrate(const TmaSet& tm, const AttnParams& p, cudaStream_t s) {
+  static std::atomic<unsigned long long> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(pp_calibrate_kernel<DPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, PcCfg::SMEM);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const dim3 grid(static_cast<unsigned>((p.nqb + 1) / 2), static_cast<unsigned>(p.H), static_cast<unsigned>(p.B));
+  pp_calibrate_kernel<DPAD><<<grid, 352, PcCfg::SMEM, s>>>(tm, p);
   return cudaGetLastError();
 }
 
