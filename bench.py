@@ -359,6 +359,26 @@ def run_ours(args, rank, world, local_rank):
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del host_in, host_out, dev_in, step_e2e
 
+    # context only: torch's fused SDPA (the pages' speed reference) on the calibration inputs
+    sdpa = None
+    try:
+        q0, k0, v0 = qkv[0]
+        for _ in range(2):
+            torch.nn.functional.scaled_dot_product_attention(q0, k0, v0)
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(3):
+            torch.nn.functional.scaled_dot_product_attention(q0, k0, v0)
+        s1.record()
+        torch.cuda.synchronize()
+        sdpa_ms = s0.elapsed_time(s1) / 3
+        sdpa_flops = 4.0 * w.L * w.L * w.d * w.B * w.H
+        sdpa = {"what": "torch.nn.functional.scaled_dot_product_attention full attention, same Q/K/V (context only)",
+                "ms": sdpa_ms, "tflops_true_L": sdpa_flops / (sdpa_ms * 1e-3) / 1e12}
+    except Exception as exc:  # noqa: BLE001
+        sdpa = {"error": str(exc)[:200]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         steps_cpu = [tuple(x.cpu() for x in qkv[0]), tuple(x.cpu() for x in qkv[1])]
@@ -382,6 +402,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline": roof(*dominant),
             "roofline_sparse_step": roof("sparse_step", sp_ms, sp_flops, sp_tf),
             "cpu_baseline": cpu,
+            "context_torch_sdpa": sdpa,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
