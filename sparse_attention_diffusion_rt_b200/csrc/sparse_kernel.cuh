@@ -8,19 +8,22 @@
 // One CTA per SM walks the (batch, head, query block) tiles tile = blockIdx.x
 // + i * gridDim.x, (batch, head) fastest (see sp_decode).  Roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
-//   warp 4     producer: validates each tile's CSR row (all lanes), then lane 0
-//              issues the TMA loads: Q (double-buffered for d <= 96), the kept
-//              K/V blocks through an NST-stage ring, and the residual tile
-//   warp 5     lane 0 issues the tcgen05 MMAs: S = Q K^T into TMEM, O += P V
-//              with P read from TMEM
+//   warp 4     producer: lane 0 validates each tile's CSR row and loads Q
+//              (double-buffered for d <= 96), the K tiles of the kept blocks
+//              and the residual tile; lane 1 loads the V tiles.  K and V have
+//              their own NST-stage rings, released after QK^T and after PV.
+//   warp 5     lane 0 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
+//              logit buffers, O += P V with P read from TMEM.  The QK^T of
+//              block j+2 is issued as soon as the softmax has read block j's
+//              logits, so the tensor pipe always has the next logits ready.
 // Tile metadata flows through a 2-slot ring (ti_*).  Every per-block barrier
 // phase is indexed by a block counter that runs across tiles, so the MMA warp
 // starts the next tile's QK^T while the softmax warps finish the previous
 // tile's epilogue; the output leaves through a shared-memory staging tile and
 // a TMA store that is only waited for when its staging slot comes round again.
 //
-// TMEM columns: S [0,128) fp32 logits, P0/P1 [128,256) bf16 probabilities,
-// O [256, 256+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
+// TMEM columns: S0/S1 [0,256) fp32 logits, P0/P1 [256,384) bf16
+// probabilities, O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
 // and every role drains what it has in flight before TMEM is freed.
 #pragma once
 #include <cuda.h>
@@ -49,7 +52,7 @@ struct SpCfg {
   static constexpr int OFF_OST = OFF_R + TILE_BYTES;
   static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static constexpr uint32_t T_S = 0, T_P0 = 128, T_P1 = 192, T_O = 256;
+  static constexpr uint32_t T_S = 0, T_P = 256, T_O = 384;   // S_b at 128b, P_b at 256 + 64b
 };
 
 struct SpTile {
@@ -59,9 +62,9 @@ struct SpTile {
 
 struct SpCtrl {
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[3], v_full[3], kv_empty[3];
-  uint64_t s_full, s_free, p_full[2];
-  uint64_t o_full, o_ready;
+  uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t o_full;
   uint64_t r_full, r_empty;
   uint64_t ti_full[2], ti_empty[2];
   uint64_t stg_ready, stg_full;
@@ -102,106 +105,102 @@ __device__ __forceinline__ void sp_decode(const AttnParams& p, int tile, int& b,
 }
 
 // ------------------------------------------------------------------ producer
+// Lane 0: tile metadata (CSR row validation), Q, K tiles, residual tile.
+// Lane 1: V tiles.  The two lanes run independent loops.
 template <int DPAD>
 __device__ __forceinline__ void sp_producer(const TmaSet& tm, const AttnParams& p, SpCtrl& ctl, uint8_t* base,
                                             int ntiles) {
   using C = SpCfg<DPAD>;
   const int lane = threadIdx.x & 31;
+  if (lane > 1) return;
   uint8_t* sQ = base + C::OFF_Q;
   uint8_t* sStage = base + C::OFF_STAGE;
   uint8_t* sR = base + C::OFF_R;
-  uint32_t g = 0, qi = 0, ri = 0;          // block, Q-load and R-load counters
-  int issued_q = 0, issued_r = 0;          // for the drain on abort
+  uint32_t g = 0, qi = 0, ri = 0;          // block, Q-load and R-load counters of this lane
   bool ok = true;
   int it = 0;
-  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int slot = it & 1;
-    if (it >= 2) {
-      ok = __all_sync(0xffffffffu, sp_wait(&ctl.ti_empty[slot], ((it >> 1) - 1) & 1, ctl, p));
-      if (!ok) break;
-    }
-    int b, h, qb;
-    sp_decode(p, tile, b, h, qb);
-    const int row = (p.Hm == 1 ? 0 : h) * p.nqb + qb;
-    int start = 0, end = 0, bad = 0;
+    int n = 0, start = 0, b = 0, h = 0, qb = 0;
     if (lane == 0) {
+      if (it >= 2 && !sp_wait(&ctl.ti_empty[slot], ((it >> 1) - 1) & 1, ctl, p)) { ok = false; break; }
+      sp_decode(p, tile, b, h, qb);
+      const int row = (p.Hm == 1 ? 0 : h) * p.nqb + qb;
       start = __ldg(p.row_ptr + row);
-      end = __ldg(p.row_ptr + row + 1);
-      if (start < 0 || end < start || static_cast<long long>(end) > p.nnz || end - start > p.nkb) bad = 1;
-    }
-    start = __shfl_sync(0xffffffffu, start, 0);
-    end = __shfl_sync(0xffffffffu, end, 0);
-    bad = __shfl_sync(0xffffffffu, bad, 0);
-    if (!bad) {
-      for (int i = lane; i < end - start; i += 32) {
-        const int c = __ldg(p.col_idx + start + i);
-        const int prev = i > 0 ? __ldg(p.col_idx + start + i - 1) : -1;
-        if (c < 0 || c >= p.nkb || c <= prev) bad = 1;
+      const int end = __ldg(p.row_ptr + row + 1);
+      int bad = (start < 0 || end < start || static_cast<long long>(end) > p.nnz || end - start > p.nkb) ? 1 : 0;
+      if (!bad) {
+        int prev = -1;
+        for (int i = start; i < end; ++i) {
+          const int c = __ldg(p.col_idx + i);
+          if (c <= prev || c >= p.nkb) { bad = 1; break; }
+          prev = c;
+        }
       }
-    }
-    bad = __any_sync(0xffffffffu, bad);
-    const int n = bad ? 0 : end - start;
-    if (lane == 0) {
-      ctl.ti[slot] = SpTile{b, h, qb, n, start, bad, -1, 128};
+      n = bad ? 0 : end - start;
+      int tail_j = -1;
+      const int tail_valid = p.L - (p.nkb - 1) * 128;
+      if (!bad && n > 0 && tail_valid < 128 && __ldg(p.col_idx + end - 1) == p.nkb - 1) tail_j = n - 1;
+      ctl.ti[slot] = SpTile{b, h, qb, n, start, bad, tail_j, tail_valid};
       if (bad) record_status(p.status, RT_ERR_BAD_INDEX);
       mbar_arrive(&ctl.ti_full[slot]);
-    }
-    __syncwarp();
-    if (bad) continue;
-    if (lane == 0) {
+      if (bad) continue;
       const int q_row = qb * 128;
       if (n > 0) {
         const int qs = C::QBUF == 2 ? (qi & 1) : 0;
         if (qi >= static_cast<uint32_t>(C::QBUF) &&
-            !sp_wait(&ctl.q_empty[qs], ((qi / C::QBUF) - 1) & 1, ctl, p)) ok = false;
-        if (ok) {
-          uint8_t* q = sQ + qs * C::TILE_BYTES;
-          mbar_arrive_expect_tx(&ctl.q_full[qs], C::TILE_BYTES);
-          tma_load_4d(q, &tm.q[0], &ctl.q_full[qs], 0, q_row, h, b);
-          if (C::C1) tma_load_4d(q + 128 * 128, &tm.q[1], &ctl.q_full[qs], 64, q_row, h, b);
-          ++qi;
-          issued_q = 1;
-        }
-        for (int j = 0; ok && j < n; ++j, ++g) {
+            !sp_wait(&ctl.q_empty[qs], ((qi / C::QBUF) - 1) & 1, ctl, p)) { ok = false; break; }
+        uint8_t* q = sQ + qs * C::TILE_BYTES;
+        mbar_arrive_expect_tx(&ctl.q_full[qs], C::TILE_BYTES);
+        tma_load_4d(q, &tm.q[0], &ctl.q_full[qs], 0, q_row, h, b);
+        if (C::C1) tma_load_4d(q + 128 * 128, &tm.q[1], &ctl.q_full[qs], 64, q_row, h, b);
+        ++qi;
+        for (int j = 0; j < n; ++j, ++g) {
           const int st = g % C::NST;
           if (g >= static_cast<uint32_t>(C::NST) &&
-              !sp_wait(&ctl.kv_empty[st], ((g / C::NST) - 1) & 1, ctl, p)) { ok = false; break; }
+              !sp_wait(&ctl.k_empty[st], ((g / C::NST) - 1) & 1, ctl, p)) { ok = false; break; }
           const int kb = __ldg(p.col_idx + start + j);
           uint8_t* sK = sStage + st * C::STAGE_BYTES;
-          uint8_t* sV = sK + C::TILE_BYTES;
           mbar_arrive_expect_tx(&ctl.k_full[st], C::TILE_BYTES);
           tma_load_4d(sK, &tm.k[0], &ctl.k_full[st], 0, kb * 128, h, b);
           if (C::C1) tma_load_4d(sK + 128 * 128, &tm.k[1], &ctl.k_full[st], 64, kb * 128, h, b);
-          mbar_arrive_expect_tx(&ctl.v_full[st], C::TILE_BYTES);
-          tma_load_4d(sV, &tm.v[0], &ctl.v_full[st], 0, kb * 128, h, b);
-          if (C::C1) tma_load_4d(sV + 128 * 128, &tm.v[1], &ctl.v_full[st], 64, kb * 128, h, b);
         }
+        if (!ok) break;
       }
-      // residual tile (bf16) for this tile's epilogue, once the previous epilogue released it
-      if (ok && !p.r_f32) {
-        if (ri >= 1 && !sp_wait(&ctl.r_empty, (ri - 1) & 1, ctl, p)) ok = false;
-        if (ok) {
-          mbar_arrive_expect_tx(&ctl.r_full, C::TILE_BYTES);
-          tma_load_4d(sR, &tm.r[0], &ctl.r_full, 0, q_row, h, b);
-          if (C::C1) tma_load_4d(sR + 128 * 128, &tm.r[1], &ctl.r_full, 64, q_row, h, b);
-          ++ri;
-          issued_r = 1;
-        }
+      if (!p.r_f32) {
+        if (ri >= 1 && !sp_wait(&ctl.r_empty, (ri - 1) & 1, ctl, p)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl.r_full, C::TILE_BYTES);
+        tma_load_4d(sR, &tm.r[0], &ctl.r_full, 0, q_row, h, b);
+        if (C::C1) tma_load_4d(sR + 128 * 128, &tm.r[1], &ctl.r_full, 64, q_row, h, b);
+        ++ri;
       }
+    } else {
+      if (!sp_wait(&ctl.ti_full[slot], (it >> 1) & 1, ctl, p)) { ok = false; break; }
+      const SpTile ti = ctl.ti[slot];
+      mbar_arrive(&ctl.ti_empty[slot]);
+      for (int j = 0; j < ti.n; ++j, ++g) {
+        const int st = g % C::NST;
+        if (g >= static_cast<uint32_t>(C::NST) &&
+            !sp_wait(&ctl.v_empty[st], ((g / C::NST) - 1) & 1, ctl, p)) { ok = false; break; }
+        const int kb = __ldg(p.col_idx + ti.start + j);
+        uint8_t* sV = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
+        mbar_arrive_expect_tx(&ctl.v_full[st], C::TILE_BYTES);
+        tma_load_4d(sV, &tm.v[0], &ctl.v_full[st], 0, kb * 128, ti.h, ti.b);
+        if (C::C1) tma_load_4d(sV + 128 * 128, &tm.v[1], &ctl.v_full[st], 64, kb * 128, ti.h, ti.b);
+      }
+      if (!ok) break;
     }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
-  if (!ok && lane == 0) {
-    // let every copy this thread started land before shared memory is released
+  if (!ok) {
+    // let every copy this lane started land before shared memory is released
     const uint64_t lim = p.wait_limit_ns;
-    if (issued_q)
+    if (lane == 0) {
       for (uint32_t i = (qi > static_cast<uint32_t>(C::QBUF) ? qi - C::QBUF : 0); i < qi; ++i)
         drain_wait(&ctl.q_full[C::QBUF == 2 ? (i & 1) : 0], (i / C::QBUF) & 1, lim);
-    if (issued_r) drain_wait(&ctl.r_full, (ri - 1) & 1, lim);
-    for (uint32_t i = (g > static_cast<uint32_t>(C::NST) ? g - C::NST : 0); i < g; ++i) {
-      drain_wait(&ctl.k_full[i % C::NST], (i / C::NST) & 1, lim);
-      drain_wait(&ctl.v_full[i % C::NST], (i / C::NST) & 1, lim);
+      if (ri >= 1) drain_wait(&ctl.r_full, (ri - 1) & 1, lim);
     }
+    for (uint32_t i = (g > static_cast<uint32_t>(C::NST) ? g - C::NST : 0); i < g; ++i)
+      drain_wait(lane == 0 ? &ctl.k_full[i % C::NST] : &ctl.v_full[i % C::NST], (i / C::NST) & 1, lim);
   }
 }
 
@@ -217,13 +216,28 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
   uint32_t g = 0, qi = 0;
   bool ok = true;
 
+  // S_(gi&1) = Q K_gi^T once the softmax has read the logits two blocks back
+  auto issue_qk = [&](uint32_t gi, uint32_t q_addr) -> bool {
+    const int st = gi % C::NST;
+    if (!sp_wait(&ctl.k_full[st], (gi / C::NST) & 1, ctl, p)) return false;
+    if (gi >= 2 && !sp_wait(&ctl.s_free[gi & 1], ((gi >> 1) - 1) & 1, ctl, p)) return false;
+    tc_fence_after();
+    const uint32_t k_tile = stage0 + st * C::STAGE_BYTES;
+    const uint32_t dst = tmem + C::T_S + 128u * (gi & 1);
+#pragma unroll
+    for (int kk = 0; kk < DPAD / 16; ++kk)
+      mma_ss(dst, kmajor_desc<DPAD>(q_addr, 128, kk), kmajor_desc<DPAD>(k_tile, 128, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+    mma_commit(&ctl.s_full[gi & 1]);
+    mma_commit(&ctl.k_empty[st]);
+    return true;
+  };
   auto issue_pv = [&](uint32_t gi, bool first) -> bool {
     const int st = gi % C::NST;
     if (!sp_wait(&ctl.p_full[gi & 1], (gi >> 1) & 1, ctl, p)) return false;
     if (!sp_wait(&ctl.v_full[st], (gi / C::NST) & 1, ctl, p)) return false;
     tc_fence_after();
     const uint32_t v_tile = stage0 + st * C::STAGE_BYTES + C::TILE_BYTES;
-    const uint32_t tp = tmem + ((gi & 1) ? C::T_P1 : C::T_P0);
+    const uint32_t tp = tmem + C::T_P + 64u * (gi & 1);
     const uint32_t dst = tmem + C::T_O;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
@@ -232,8 +246,8 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
       if (C::C1 > 0 && DPAD != 128)
         mma_ts(dst + 64, tp + kk * 8, v_desc_c1<DPAD, 128>(v_tile, kk), IDESC_PV_C1, acc);
     }
-    mma_commit(&ctl.kv_empty[st]);
-    mma_commit(&ctl.o_ready);
+    mma_commit(&ctl.v_empty[st]);
+    mma_commit(&ctl.pv_done[gi & 1]);
     return true;
   };
 
@@ -246,23 +260,17 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
       const int qs = C::QBUF == 2 ? (qi & 1) : 0;
       if (!sp_wait(&ctl.q_full[qs], (qi / C::QBUF) & 1, ctl, p)) { ok = false; break; }
       const uint32_t q_addr = q0 + qs * C::TILE_BYTES;
-      for (int j = 0; j < n; ++j, ++g) {
-        const int st = g % C::NST;
-        if (!sp_wait(&ctl.k_full[st], (g / C::NST) & 1, ctl, p)) { ok = false; break; }
-        if (g > 0 && !sp_wait(&ctl.s_free, (g - 1) & 1, ctl, p)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_tile = stage0 + st * C::STAGE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < DPAD / 16; ++kk)
-          mma_ss(tmem + C::T_S, kmajor_desc<DPAD>(q_addr, 128, kk), kmajor_desc<DPAD>(k_tile, 128, kk),
-                 IDESC_QK, kk > 0 ? 1u : 0u);
-        mma_commit(&ctl.s_full);
-        if (j == n - 1) mma_commit(&ctl.q_empty[qs]);
-        if (j > 0 && !issue_pv(g - 1, j == 1)) { ok = false; break; }
+      const uint32_t g0 = g;
+      for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_qk(g0 + i, q_addr);
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 2 < n) ok = issue_qk(g0 + j + 2, q_addr);
+        if (ok && j + 2 == n) mma_commit(&ctl.q_empty[qs]);   // the tile's last QK^T has been issued
+        if (ok) ok = issue_pv(g0 + j, j == 0);
       }
       if (!ok) break;
-      if (!issue_pv(g - 1, n == 1)) { ok = false; break; }
+      if (n == 1) mma_commit(&ctl.q_empty[qs]);
       mma_commit(&ctl.o_full);
+      g = g0 + n;
       ++qi;
     }
     mbar_arrive(&ctl.ti_empty[slot]);
@@ -301,16 +309,16 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
     const float rho = grow < p.L ? __ldg(p.rho_in + rho_idx) : 0.f;
     float m = 0.f, l = 0.f;
     for (int j = 0; j < ti.n; ++j, ++g) {
-      ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full, g & 1, ctl, p));
+      const int bf = g & 1;
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full[bf], (g >> 1) & 1, ctl, p));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
-      load_scores<128>(tS, s);
+      load_scores<128>(tS + 128u * bf, s);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&ctl.s_free);
-      const int kb = __ldg(p.col_idx + ti.start + j);
-      mask_tail<128>(s, p.L - kb * 128);
+      mbar_arrive(&ctl.s_free[bf]);
+      mask_tail<128>(s, (j == ti.tail_j) ? ti.tail_valid : 128);
       const float mx = row_max<128>(s) * sl2;
       if (j == 0) {
         m = mx;
@@ -318,17 +326,23 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
         const float m_new = fmaxf(m, mx);
         const float alpha = ex2_approx(m - m_new);
         l *= alpha;
-        ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_ready, (g - 1) & 1, ctl, p));
+        // O holds blocks up to g-1: wait for PV(g-1)
+        ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, ctl, p));
         if (!ok) break;
         tc_fence_after();
         rescale_row<DPAD>(tO, alpha);
         m = m_new;
       }
-      const uint32_t tP = tmem + lane_base + ((g & 1) ? C::T_P1 : C::T_P0);
-      l += exp_pack_store<128>(s, sl2, m, tP);
+      // P buffer bf was last read by PV(g-2)
+      if (g >= 2) {
+        ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[bf], ((g >> 1) - 1) & 1, ctl, p));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      l += exp_pack_store<128>(s, sl2, m, tmem + lane_base + C::T_P + 64u * bf);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ctl.p_full[g & 1]);
+      mbar_arrive(&ctl.p_full[bf]);
     }
     if (!ok) break;
     // ------------------------------------------------------------- epilogue
@@ -433,19 +447,20 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.q_full[i], 1);
       mbar_init(&ctl.q_empty[i], 1);
+      mbar_init(&ctl.s_full[i], 1);
+      mbar_init(&ctl.s_free[i], kSoftmaxThreads);
       mbar_init(&ctl.p_full[i], kSoftmaxThreads);
+      mbar_init(&ctl.pv_done[i], 1);
       mbar_init(&ctl.ti_full[i], 1);
-      mbar_init(&ctl.ti_empty[i], kSoftmaxThreads + 1);
+      mbar_init(&ctl.ti_empty[i], kSoftmaxThreads + 2);
     }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&ctl.k_full[i], 1);
       mbar_init(&ctl.v_full[i], 1);
-      mbar_init(&ctl.kv_empty[i], 1);
+      mbar_init(&ctl.k_empty[i], 1);
+      mbar_init(&ctl.v_empty[i], 1);
     }
-    mbar_init(&ctl.s_full, 1);
-    mbar_init(&ctl.s_free, kSoftmaxThreads);
     mbar_init(&ctl.o_full, 1);
-    mbar_init(&ctl.o_ready, 1);
     mbar_init(&ctl.r_full, 1);
     mbar_init(&ctl.r_empty, kSoftmaxThreads);
     mbar_init(&ctl.stg_ready, 1);
