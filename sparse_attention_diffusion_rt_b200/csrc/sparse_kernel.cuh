@@ -6,7 +6,7 @@
 // plus the cached residual of the masked tokens; reply to Pwod's W1: ramp-up).
 //
 // One CTA per SM walks the (batch, head, query block) tiles tile = blockIdx.x
-// + i * gridDim.x, (batch, head) fastest (see sp_decode).  Roles (192 threads):
+// + i * gridDim.x, query block fastest (see sp_decode).  Roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
 //   warp 4     producer: lane 0 validates each tile's CSR row and loads Q
 //              (double-buffered for d <= 96), the K tiles of the kept blocks
@@ -93,13 +93,14 @@ __device__ __forceinline__ bool sp_wait(uint64_t* bar, uint32_t parity, CtrlT& c
   }
 }
 
-// Tile order: (batch, head) fastest, then query block.  Concurrent CTAs then
-// spread over many heads, so key blocks that every query block keeps (text
-// tokens) are not fetched by every SM at once, while each head's local key
-// blocks are still shared in L2 by the few neighbouring query blocks in flight.
+// Tile order: query block fastest within a (batch, head).  The CTAs in flight
+// then cover a contiguous range of query blocks of one head, whose kept key
+// blocks (local windows) overlap, so each K/V block is fetched from DRAM about
+// once and re-read from L2.  (A (batch, head)-fastest order measured 8x the
+// compulsory DRAM traffic on the long-video masks: reuse distance beyond L2.)
 __device__ __forceinline__ void sp_decode(const AttnParams& p, int tile, int& b, int& h, int& qb) {
-  const int bh = tile % (p.B * p.H);
-  qb = tile / (p.B * p.H);
+  qb = tile % p.nqb;
+  const int bh = tile / p.nqb;
   b = bh / p.H;
   h = bh % p.H;
 }
