@@ -9,6 +9,7 @@
 #include "sparse_kernel.cuh"
 #include "pp_sparse.cuh"
 #include "pp_calibrate.cuh"
+#include "cal_kernel.cuh"
 
 namespace rtb {
 
@@ -50,6 +51,26 @@ cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, c
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  kern<<<grid, kThreads, smem, s>>>(tm, p);
+  return cudaGetLastError();
+}
+
+// Calibration kernel with one TMEM accumulator (d > 64, 128-token blocks):
+// one CTA per (query block, head, batch).
+template <int DPAD>
+cudaError_t launch_cal_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, cudaStream_t s) {
+  auto kern = cal_kernel<DPAD>;
+  constexpr int smem = CalCfg<DPAD>::SMEM > kMinSmem ? CalCfg<DPAD>::SMEM : kMinSmem;
+  static std::atomic<unsigned long long> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
