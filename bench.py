@@ -48,7 +48,7 @@ from sparse_attention_diffusion_rt_b200 import inputs  # noqa: E402
 METRIC = "sparse-step attention latency & TFLOP/s (executed blocks), % bf16 peak, 1 B200"
 DEFAULT_WORKLOAD = "longvideo-3.1"
 KERNEL_SOURCES = ("attn_kernel.cuh", "ptx.cuh", "softmax.cuh", "sparse_kernel.cuh", "pp_sparse.cuh",
-                  "pp_calibrate.cuh", "attn_launch.h")
+                  "pp_calibrate.cuh", "cal_kernel.cuh", "attn_launch.h")
 
 
 # ---------------------------------------------------------------------------

@@ -5,19 +5,24 @@
 // full attention, the denominator ratio rho = Z_sparse / Z_full and the
 // residual of the masked tokens, all under one shared row max):
 //   O = (acc_in + acc_out) / Z,  R = acc_out / Z,  rho = l_in / Z,  Z = l_in + l_out.
-// Instead of two TMEM accumulators, every CTA visits its key blocks in the
-// order "masked blocks (ascending), then kept blocks (ascending)".  When the
-// first kept block is reached, the accumulator (then exactly acc_out) is copied
-// to shared memory as fp32 and the accumulation restarts at zero; later lazy
+// Instead of two accumulators, every CTA visits its key blocks in the order
+// "masked blocks (ascending), then kept blocks (ascending)".  When the first
+// kept block is reached, the accumulator (then exactly acc_out) is copied to
+// spare TMEM columns and the accumulation restarts at zero; later lazy
 // rescalings of the running max multiply that copy by a per-row factor.  The
 // sums do not depend on the visiting order, so the result is the same
-// definition; the freed TMEM pays for double-buffered logits and
-// probabilities: S0/S1 [0,256) fp32, P0/P1 [256,384) bf16, acc [384,384+DPAD).
+// definition.
+//
+// TMEM columns: S0/S1 [0,256) fp32 logits, each with its bf16 probabilities P
+// written over its first 64 columns once the logits are in registers; the
+// accumulator [256, 256+DPAD); the masked-block copy [384, 384+DPAD).  With no
+// P or copy in shared memory, the K and V rings get as many stages as fit.
 //
 // One CTA per (batch, head, query block), 192 threads: warps 0-3 softmax and
 // epilogue (thread t owns row t), warp 4 lane 0 loads Q and the K tiles, lane 1
-// the V tiles (separate rings), warp 5 lane 0 issues the MMAs; the QK^T of
-// block j+2 is issued as soon as the softmax has read block j's logits.
+// the V tiles, warp 5 lane 0 issues the MMAs in the order PV(j), QK(j+2): the
+// logits of block j+2 overwrite P(j), and MMAs of one thread execute in issue
+// order, so the softmax never waits for a buffer, only for its logits.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -33,20 +38,20 @@ template <int DPAD>
 struct CalCfg {
   static constexpr int C1 = DPAD - 64;
   static constexpr int TILE = 128 * DPAD * 2;
-  static constexpr int NST = DPAD <= 96 ? 3 : 2;
-  static constexpr int SNAP_ROW = DPAD * 4;                  // fp32 row of the snapshot
   static constexpr int OFF_Q = 2048;
   static constexpr int OFF_STAGE = OFF_Q + TILE;
-  static constexpr int OFF_SNAP = OFF_STAGE + NST * 2 * TILE;
-  static constexpr int SMEM = OFF_SNAP + 128 * SNAP_ROW + 1024;
+  static constexpr int NST_FIT = (232448 - 1024 - OFF_STAGE) / (2 * TILE);
+  static constexpr int NST = NST_FIT > 6 ? 6 : NST_FIT;
+  static constexpr int SMEM = OFF_STAGE + NST * 2 * TILE + 1024;
+  static_assert(NST >= 2, "at least two K/V stages");
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static_assert(NST * 2 * TILE >= 128 * ((DPAD + 31) / 32) * 128, "residual staging fits the stages");
-  static constexpr uint32_t T_S = 0, T_P = 256, T_ACC = 384;
+  static constexpr uint32_t T_S = 0, T_ACC = 256, T_SNAP = 384;
 };
 
 struct CalCtrl {
-  uint64_t q_full, s_full[2], s_free[2], p_full[2], pv_done[2], o_full, epi, drain;
-  uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
+  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, epi, drain;
+  uint64_t k_full[6], v_full[6], k_empty[6], v_empty[6];
   uint32_t tmem_base;
   volatile int abort_flag;
   int bad_index;
@@ -118,10 +123,10 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
   const int n = p.nkb;
   const int n_masked = p.nkb - ctl.n_kept;
 
+  // S_(j&1) = Q K_j^T.  For j >= 2 it overwrites P(j-2), whose PV was issued before.
   auto issue_qk = [&](int j) -> bool {
     const int st = j % C::NST;
     if (!sp_wait(&ctl.k_full[st], (j / C::NST) & 1, ctl, p)) return false;
-    if (j >= 2 && !sp_wait(&ctl.s_free[j & 1], ((j >> 1) - 1) & 1, ctl, p)) return false;
     tc_fence_after();
     const uint32_t k_tile = stage0 + st * 2 * C::TILE;
 #pragma unroll
@@ -138,9 +143,9 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
     if (!sp_wait(&ctl.v_full[st], (j / C::NST) & 1, ctl, p)) return false;
     tc_fence_after();
     const uint32_t v_tile = stage0 + st * 2 * C::TILE + C::TILE;
-    const uint32_t tp = tmem + C::T_P + 64u * (j & 1);
+    const uint32_t tp = tmem + C::T_S + 128u * (j & 1);
     const uint32_t dst = tmem + C::T_ACC;
-    const bool first = (j == 0) || (j == n_masked);     // restart after the snapshot
+    const bool first = (j == 0) || (j == n_masked);     // restart after the copy of the masked blocks
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint32_t acc = (first && kk == 0) ? 0u : 1u;
@@ -155,8 +160,8 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
 
   bool ok = sp_wait(&ctl.q_full, 0, ctl, p) && issue_qk(0) && (n < 2 || issue_qk(1));
   for (int j = 0; ok && j < n; ++j) {
-    if (j + 2 < n && !issue_qk(j + 2)) { ok = false; break; }
     if (!issue_pv(j)) { ok = false; break; }
+    if (j + 2 < n && !issue_qk(j + 2)) { ok = false; break; }
   }
   if (ok) {
     mma_commit(&ctl.o_full);
@@ -174,28 +179,29 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
   const uint32_t lane_base = static_cast<uint32_t>((t >> 5) * 32) << 16;
   const uint32_t tl = tmem + lane_base;
   const uint32_t tAcc = tl + C::T_ACC;
-  float* snap = reinterpret_cast<float*>(base + C::OFF_SNAP);
+  const uint32_t tSnap = tl + C::T_SNAP;
   const float sl2 = p.scale_log2;
   const int n = p.nkb;
   const int n_masked = p.nkb - ctl.n_kept;
-  const bool split = n_masked > 0 && ctl.n_kept > 0;    // a snapshot is taken between the phases
-  CalOrder order{0, n_masked == 0 ? 1 : 0};
+  const bool split = n_masked > 0 && ctl.n_kept > 0;    // a copy is taken between the phases
+  // the last key block (the one that may run past the sequence end) is the
+  // last of its phase in the visiting order
+  const bool tail_kept = (ctl.kept_bits[(p.nkb - 1) >> 5] >> ((p.nkb - 1) & 31)) & 1u;
+  const int tail_j = tail_kept ? n - 1 : n_masked - 1;
+  const int tail_valid = p.L - (p.nkb - 1) * 128;
   float m = 0.f, l_in = 0.f, l_out = 0.f, snap_scale = 1.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
     const int bf = j & 1;
-    const int kb = order.next(ctl, p.nkb);
     ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full[bf], (j >> 1) & 1, ctl, p));
     if (!ok) break;
     tc_fence_after();
+    const uint32_t tS = tl + C::T_S + 128u * bf;
     uint32_t s[128];
-    load_scores<128>(tl + C::T_S + 128u * bf, s);
+    load_scores<128>(tS, s);
     tmem_wait_ld();
-    tc_fence_before();
-    mbar_arrive(&ctl.s_free[bf]);
-    mask_tail<128>(s, p.L - kb * 128);
+    if (j == tail_j) mask_tail<128>(s, tail_valid);
     const float mx = row_max<128>(s) * sl2;
-    bool acc_ready = false;                   // PV(j-1) known complete
     if (j == 0) {
       m = mx;
     } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
@@ -204,44 +210,33 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
       l_in *= alpha;
       l_out *= alpha;
       if (split && j >= n_masked) snap_scale *= alpha;   // the copy is relative to the old max
+      // the accumulator holds blocks 0..j-1: wait until the last of them has landed
       ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl, p));
       if (!ok) break;
-      acc_ready = true;
       tc_fence_after();
-      // right after the snapshot the accumulator restarts, so only rescale what it holds
+      // at the first kept block the accumulator is copied and restarted: nothing to rescale
       if (!(split && j == n_masked)) rescale_row<DPAD>(tAcc, alpha);
       m = m_new;
     }
     if (split && j == n_masked) {
-      // the accumulator now holds exactly the masked blocks: keep it in shared memory
-      if (!acc_ready) {
-        ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl, p));
-        if (!ok) break;
-        tc_fence_after();
-      }
+      // the accumulator now holds exactly the masked blocks: copy it to its own columns
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl, p));
+      if (!ok) break;
+      tc_fence_after();
+      const float sc = snap_scale;            // 1, or the rescale taken at this very block
 #pragma unroll
       for (int c = 0; c < DPAD; c += 16) {
         uint32_t a[16];
         tmem_ld_x16(tAcc + c, a);
         tmem_wait_ld();
-        const float sc = snap_scale;          // 1, or the rescale taken at this very block
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 v4 = make_float4(__uint_as_float(a[4 * u]) * sc, __uint_as_float(a[4 * u + 1]) * sc,
-                                        __uint_as_float(a[4 * u + 2]) * sc, __uint_as_float(a[4 * u + 3]) * sc);
-          const int unit = ((c >> 2) + u + t) % (DPAD / 4);   // rotate 16-byte units by row
-          *reinterpret_cast<float4*>(snap + t * DPAD + unit * 4) = v4;
-        }
+        for (int i = 0; i < 16; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * sc);
+        tmem_st_x16(tSnap + c, a);
       }
       snap_scale = 1.f;
     }
-    // P buffer bf was last read by PV(j-2)
-    if (j >= 2) {
-      ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[bf], ((j >> 1) - 1) & 1, ctl, p));
-      if (!ok) break;
-      tc_fence_after();
-    }
-    const float sum = exp_pack_store<128>(s, sl2, m, tl + C::T_P + 64u * bf);
+    // P(j) over the first 64 logit columns: the logits are in registers
+    const float sum = exp_pack_store<128>(s, sl2, m, tS);
     if (j < n_masked) l_out += sum; else l_in += sum;
     tmem_wait_st();
     tc_fence_before();
@@ -262,36 +257,27 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     const float rs = snap_scale * inv;
 #pragma unroll
     for (int c = 0; c < DPAD; c += 16) {
-      uint32_t a[16];
+      uint32_t a[16], sv[16];
       tmem_ld_x16(tAcc + c, a);
+      if (split) tmem_ld_x16(tSnap + c, sv);
       tmem_wait_ld();
       float o16[16], r16[16];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float4 sv = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < 16; ++i) {
+        const float acc = __uint_as_float(a[i]);
+        float out_masked, out_kept;
         if (split) {
-          const int unit = ((c >> 2) + u + t) % (DPAD / 4);
-          sv = *reinterpret_cast<const float4*>(snap + t * DPAD + unit * 4);
+          out_masked = __uint_as_float(sv[i]) * rs;
+          out_kept = acc * inv;
+        } else if (n_masked == 0) {
+          out_masked = 0.f;
+          out_kept = acc * inv;
+        } else {                                 // no kept block: the accumulator is all masked
+          out_masked = acc * inv;
+          out_kept = 0.f;
         }
-        const float sr[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * u + e;
-          const float acc = __uint_as_float(a[i]);
-          float out_masked, out_kept;
-          if (split) {
-            out_masked = sr[e] * rs;
-            out_kept = acc * inv;
-          } else if (n_masked == 0) {
-            out_masked = 0.f;
-            out_kept = acc * inv;
-          } else {                                 // no kept block: the accumulator is all masked
-            out_masked = acc * inv;
-            out_kept = 0.f;
-          }
-          o16[i] = out_masked + out_kept;
-          r16[i] = out_masked;
-        }
+        o16[i] = out_masked + out_kept;
+        r16[i] = out_masked;
       }
       store_row16<DPAD>(sO, 128, t, c, false, o16);
       store_row16<DPAD>(sRst, 128, t, c, p.r_f32 != 0, r16);
@@ -332,11 +318,10 @@ cal_kernel(const __grid_constant__ TmaSet tm, const AttnParams p) {
     mbar_init(&ctl.q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.s_full[i], 1);
-      mbar_init(&ctl.s_free[i], kSoftmaxThreads);
       mbar_init(&ctl.p_full[i], kSoftmaxThreads);
       mbar_init(&ctl.pv_done[i], 1);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < C::NST; ++i) {
       mbar_init(&ctl.k_full[i], 1);
       mbar_init(&ctl.v_full[i], 1);
       mbar_init(&ctl.k_empty[i], 1);
