@@ -87,6 +87,21 @@ def profiled_traffic(kernel_tag: str, workload: str):
     return float(m_bytes.group(1))
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (one all-reduce; every rank must call it)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput of weak-scaled replicas: every rank does the same
+    work per step, and a step lasts as long as the slowest rank's."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
 
@@ -306,12 +321,9 @@ def run_ours(args, rank, world, local_rank):
     st = rt.rt_check_device_error()
     if st != 0:
         raise RuntimeError(f"device error in timed region: {rt.rt_status_string(st)}")
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(world, step_flops, ms_per_step)
 
     # ---- per-kernel timing: separate pass, each kernel bracketed by events
     step.times = {"calibrate": [], "sparse": []}
@@ -369,11 +381,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, world, dev)
+        e2e = {"value": job_tflops(world, step_flops, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del host_in, host_out, dev_in, step_e2e
 
