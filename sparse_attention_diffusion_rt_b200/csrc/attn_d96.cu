@@ -6,7 +6,7 @@ namespace rtb {
 cudaError_t launch_attn_d96(bool cal, int block, const TmaSet& tm, const AttnParams& p, dim3 grid,
                            cudaStream_t s) {
   if (block != 128) return cudaErrorInvalidValue;
-  return cal ? launch_cal_impl<96>(tm, p, grid, s) : launch_sparse_impl<96>(tm, p, s);
+  return cal ? launch_cal_impl<96, true>(tm, p, grid, s) : launch_sparse_impl<96>(tm, p, s);
 }
 
 }  // namespace rtb

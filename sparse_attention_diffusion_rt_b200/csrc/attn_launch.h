@@ -59,11 +59,11 @@ cudaError_t launch_attn_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, c
 }
 
 // Calibration kernel with one TMEM accumulator (d > 64, 128-token blocks):
-// one CTA per (query block, head, batch).
-template <int DPAD>
+// one CTA per (query block, head, batch); QT = Q in TMEM.
+template <int DPAD, bool QT>
 cudaError_t launch_cal_impl(const TmaSet& tm, const AttnParams& p, dim3 grid, cudaStream_t s) {
-  auto kern = cal_kernel<DPAD>;
-  constexpr int smem = CalCfg<DPAD>::SMEM > kMinSmem ? CalCfg<DPAD>::SMEM : kMinSmem;
+  auto kern = cal_kernel<DPAD, QT>;
+  constexpr int smem = CalCfg<DPAD, QT>::SMEM > kMinSmem ? CalCfg<DPAD, QT>::SMEM : kMinSmem;
   static std::atomic<unsigned long long> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

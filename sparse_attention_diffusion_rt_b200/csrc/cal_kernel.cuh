@@ -15,8 +15,14 @@
 //
 // TMEM columns: S0/S1 [0,256) fp32 logits, each with its bf16 probabilities P
 // written over its first 64 columns once the logits are in registers; the
-// accumulator [256, 256+DPAD); the masked-block copy [384, 384+DPAD).  With no
-// P or copy in shared memory, the K and V rings get as many stages as fit.
+// accumulator [256, 256+DPAD); then the masked-block copy.  With QT (Q in
+// TMEM) the copy follows the accumulator and Q follows the copy as bf16 pairs,
+// so that QK^T takes A from TMEM and shared memory carries only K and V to
+// the tensor core (the operand traffic that bounds this kernel).  At DPAD = 128
+// the copy then has to fit 64 columns: it is stored as f16 pairs with a
+// power-of-two row scale chosen from the row's largest value (relative error
+// below 2^-11 of that value); without QT it is fp32 at [384, 512).  With no P
+// or copy in shared memory, the K and V rings get as many stages as fit.
 //
 // One CTA per (batch, head, query block), 192 threads: warps 0-3 softmax and
 // epilogue (thread t owns row t), warp 4 lane 0 loads Q and the K tiles, lane 1
@@ -34,7 +40,7 @@
 
 namespace rtb {
 
-template <int DPAD>
+template <int DPAD, bool QT>
 struct CalCfg {
   static constexpr int C1 = DPAD - 64;
   static constexpr int TILE = 128 * DPAD * 2;
@@ -46,11 +52,16 @@ struct CalCfg {
   static_assert(NST >= 2, "at least two K/V stages");
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static_assert(NST * 2 * TILE >= 128 * ((DPAD + 31) / 32) * 128, "residual staging fits the stages");
-  static constexpr uint32_t T_S = 0, T_ACC = 256, T_SNAP = 384;
+  static constexpr bool SNAP16 = QT && DPAD == 128;          // f16 copy with a row scale
+  static constexpr uint32_t T_S = 0, T_ACC = 256;
+  static constexpr uint32_t T_SNAP = QT ? 256 + DPAD : 384;
+  static constexpr uint32_t SNAP_COLS = SNAP16 ? DPAD / 2 : DPAD;
+  static constexpr uint32_t T_Q = T_SNAP + SNAP_COLS;          // QT: Q as bf16 pairs, DPAD / 2 columns
+  static_assert(T_SNAP + SNAP_COLS <= 512 && (!QT || T_Q + DPAD / 2 <= 512), "TMEM columns");
 };
 
 struct CalCtrl {
-  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, epi, drain;
+  uint64_t q_full, q_tmem, s_full[2], p_full[2], pv_done[2], o_full, epi, drain;
   uint64_t k_full[6], v_full[6], k_empty[6], v_empty[6];
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -77,10 +88,10 @@ struct CalOrder {
   }
 };
 
-template <int DPAD>
+template <int DPAD, bool QT>
 __device__ __forceinline__ void cal_producer(const TmaSet& tm, const AttnParams& p, CalCtrl& ctl, uint8_t* base,
                                              int b, int h, int qb) {
-  using C = CalCfg<DPAD>;
+  using C = CalCfg<DPAD, QT>;
   const int lane = threadIdx.x & 31;
   if (lane > 1) return;
   int issued = 0;
@@ -112,9 +123,9 @@ __device__ __forceinline__ void cal_producer(const TmaSet& tm, const AttnParams&
   }
 }
 
-template <int DPAD>
+template <int DPAD, bool QT>
 __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8_t* base, uint32_t tmem) {
-  using C = CalCfg<DPAD>;
+  using C = CalCfg<DPAD, QT>;
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t IDESC_PV_FULL = make_idesc_bf16(128, DPAD == 128 ? 128 : 64, 0, 1);
   constexpr uint32_t IDESC_PV_C1 = make_idesc_bf16(128, C::C1 > 0 ? C::C1 : 16, 0, 1);
@@ -130,9 +141,14 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
     tc_fence_after();
     const uint32_t k_tile = stage0 + st * 2 * C::TILE;
 #pragma unroll
-    for (int kk = 0; kk < DPAD / 16; ++kk)
-      mma_ss(tmem + C::T_S + 128u * (j & 1), kmajor_desc<DPAD>(q_addr, 128, kk), kmajor_desc<DPAD>(k_tile, 128, kk),
-             IDESC_QK, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < DPAD / 16; ++kk) {
+      if constexpr (QT)
+        mma_ts(tmem + C::T_S + 128u * (j & 1), tmem + C::T_Q + kk * 8, kmajor_desc<DPAD>(k_tile, 128, kk), IDESC_QK,
+               kk > 0 ? 1u : 0u);
+      else
+        mma_ss(tmem + C::T_S + 128u * (j & 1), kmajor_desc<DPAD>(q_addr, 128, kk),
+               kmajor_desc<DPAD>(k_tile, 128, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+    }
     mma_commit(&ctl.s_full[j & 1]);
     mma_commit(&ctl.k_empty[st]);
     return true;
@@ -158,7 +174,8 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
     return true;
   };
 
-  bool ok = sp_wait(&ctl.q_full, 0, ctl, p) && issue_qk(0) && (n < 2 || issue_qk(1));
+  // Q in TMEM: the softmax warps copy it there from shared memory first
+  bool ok = sp_wait(QT ? &ctl.q_tmem : &ctl.q_full, 0, ctl, p) && issue_qk(0) && (n < 2 || issue_qk(1));
   for (int j = 0; ok && j < n; ++j) {
     if (!issue_pv(j)) { ok = false; break; }
     if (j + 2 < n && !issue_qk(j + 2)) { ok = false; break; }
@@ -171,10 +188,31 @@ __device__ __forceinline__ void cal_mma(const AttnParams& p, CalCtrl& ctl, uint8
   }
 }
 
-template <int DPAD>
+// Q row t (bf16, as TMA left it in the swizzled chunks) -> TMEM lane t as bf16
+// pairs, the A-operand layout of QK^T.
+template <int DPAD, bool QT>
+__device__ __forceinline__ void cal_copy_q(const uint8_t* sQ, uint32_t tq, int t) {
+  using C = CalCfg<DPAD, QT>;
+#pragma unroll
+  for (int u0 = 0; u0 < DPAD / 8; u0 += 2) {          // two 16-byte units (16 columns) per store
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int u = u0 + k;
+      const bool c1 = u >= 8;
+      const uint32_t rb = c1 ? C::C1 * 2 : 128;
+      const uint32_t off = (c1 ? 128 * 128 : 0) + swz_off(t * rb + (c1 ? u - 8 : u) * 16, rb);
+      const uint4 v = *reinterpret_cast<const uint4*>(sQ + off);
+      w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+    }
+    tmem_st_x8(tq + u0 * 4, w);
+  }
+}
+
+template <int DPAD, bool QT>
 __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& p, CalCtrl& ctl, uint8_t* base,
                                             uint32_t tmem, int b, int h, int qb) {
-  using C = CalCfg<DPAD>;
+  using C = CalCfg<DPAD, QT>;
   const int t = threadIdx.x;
   const uint32_t lane_base = static_cast<uint32_t>((t >> 5) * 32) << 16;
   const uint32_t tl = tmem + lane_base;
@@ -191,7 +229,16 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
   const int tail_valid = p.L - (p.nkb - 1) * 128;
   float m = 0.f, l_in = 0.f, l_out = 0.f, snap_scale = 1.f;
   bool ok = true;
-  for (int j = 0; j < n; ++j) {
+  if constexpr (QT) {
+    ok = __all_sync(0xffffffffu, sp_wait(&ctl.q_full, 0, ctl, p));
+    if (ok) {
+      cal_copy_q<DPAD, QT>(base + C::OFF_Q, tl + C::T_Q, t);
+      tmem_wait_st();
+      tc_fence_before();
+    }
+    mbar_arrive(&ctl.q_tmem);
+  }
+  for (int j = 0; ok && j < n; ++j) {
     const int bf = j & 1;
     ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full[bf], (j >> 1) & 1, ctl, p));
     if (!ok) break;
@@ -201,11 +248,16 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     load_scores<128>(tS, s);
     tmem_wait_ld();
     if (j == tail_j) mask_tail<128>(s, tail_valid);
-    const float mx = row_max<128>(s) * sl2;
-    if (j == 0) {
-      m = mx;
-    } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
-      const float m_new = fmaxf(m, mx);
+    if (j == 0) m = row_max<128>(s) * sl2;
+    // P(j) over the first 64 logit columns (the logits are in registers), with
+    // the running max; xmax, the block's largest x = s * sl2 - m, tells whether
+    // that max was too small
+    float xmax;
+    float sum = exp_pack_store_mx<128>(s, sl2, m, tS, xmax);
+    if (__any_sync(0xffffffffu, xmax > kRescaleLog2)) {
+      // rare: the block raised the max by more than 2^8: rescale, then redo P(j)
+      tmem_wait_st();                         // the first P(j) stores land before they are redone
+      const float m_new = m + fmaxf(xmax, 0.f);
       const float alpha = ex2_approx(m - m_new);
       l_in *= alpha;
       l_out *= alpha;
@@ -217,6 +269,7 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
       // at the first kept block the accumulator is copied and restarted: nothing to rescale
       if (!(split && j == n_masked)) rescale_row<DPAD>(tAcc, alpha);
       m = m_new;
+      sum = exp_pack_store<128>(s, sl2, m, tS);
     }
     if (split && j == n_masked) {
       // the accumulator now holds exactly the masked blocks: copy it to its own columns
@@ -224,19 +277,45 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
       if (!ok) break;
       tc_fence_after();
       const float sc = snap_scale;            // 1, or the rescale taken at this very block
+      if constexpr (C::SNAP16) {
+        // f16 with a power-of-two row scale: the row's largest |value| lands in [2^14, 2^15)
+        float amax = 0.f;
 #pragma unroll
-      for (int c = 0; c < DPAD; c += 16) {
-        uint32_t a[16];
-        tmem_ld_x16(tAcc + c, a);
-        tmem_wait_ld();
+        for (int c = 0; c < DPAD; c += 16) {
+          uint32_t a[16];
+          tmem_ld_x16(tAcc + c, a);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * sc);
-        tmem_st_x16(tSnap + c, a);
+          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(a[i])));
+        }
+        int e = 0;
+        frexpf(amax * sc, &e);                // amax * sc = f * 2^e, f in [0.5, 1)
+        const int k = min(15 - e, 126);
+        const float f = sc * __int_as_float((127 + k) << 23);    // sc * 2^k
+#pragma unroll
+        for (int c = 0; c < DPAD; c += 16) {
+          uint32_t a[16], w[8];
+          tmem_ld_x16(tAcc + c, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            w[i] = pack_f16x2(__uint_as_float(a[2 * i]) * f, __uint_as_float(a[2 * i + 1]) * f);
+          tmem_st_x8(tSnap + c / 2, w);
+        }
+        snap_scale = __int_as_float((127 - k) << 23);           // 2^-k
+      } else {
+#pragma unroll
+        for (int c = 0; c < DPAD; c += 16) {
+          uint32_t a[16];
+          tmem_ld_x16(tAcc + c, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * sc);
+          tmem_st_x16(tSnap + c, a);
+        }
+        snap_scale = 1.f;
       }
-      snap_scale = 1.f;
     }
-    // P(j) over the first 64 logit columns: the logits are in registers
-    const float sum = exp_pack_store<128>(s, sl2, m, tS);
     if (j < n_masked) l_out += sum; else l_in += sum;
     tmem_wait_st();
     tc_fence_before();
@@ -259,7 +338,22 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     for (int c = 0; c < DPAD; c += 16) {
       uint32_t a[16], sv[16];
       tmem_ld_x16(tAcc + c, a);
-      if (split) tmem_ld_x16(tSnap + c, sv);
+      if constexpr (C::SNAP16) {
+        if (split) {
+          uint32_t w[8];
+          tmem_ld_x8(tSnap + c / 2, w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float lo, hi;
+            unpack_f16x2(w[i], lo, hi);
+            sv[2 * i] = __float_as_uint(lo);
+            sv[2 * i + 1] = __float_as_uint(hi);
+          }
+        }
+      } else {
+        if (split) tmem_ld_x16(tSnap + c, sv);
+      }
       tmem_wait_ld();
       float o16[16], r16[16];
 #pragma unroll
@@ -302,10 +396,10 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
   }
 }
 
-template <int DPAD>
+template <int DPAD, bool QT>
 __global__ void __launch_bounds__(kThreads, 1)
 cal_kernel(const __grid_constant__ TmaSet tm, const AttnParams p) {
-  using C = CalCfg<DPAD>;
+  using C = CalCfg<DPAD, QT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -316,6 +410,7 @@ cal_kernel(const __grid_constant__ TmaSet tm, const AttnParams p) {
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.q_full, 1);
+    mbar_init(&ctl.q_tmem, kSoftmaxThreads);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.s_full[i], 1);
       mbar_init(&ctl.p_full[i], kSoftmaxThreads);
@@ -371,11 +466,11 @@ cal_kernel(const __grid_constant__ TmaSet tm, const AttnParams p) {
   if (ctl.bad_index) {
     if (threadIdx.x == 0) record_status(p.status, RT_ERR_BAD_INDEX);
   } else if (warp == kProducerWarp) {
-    cal_producer<DPAD>(tm, p, ctl, base, b, h, qb);
+    cal_producer<DPAD, QT>(tm, p, ctl, base, b, h, qb);
   } else if (warp == kMmaWarp) {
-    if (lane == 0) cal_mma<DPAD>(p, ctl, base, tmem);
+    if (lane == 0) cal_mma<DPAD, QT>(p, ctl, base, tmem);
   } else {
-    cal_softmax<DPAD>(tm, p, ctl, base, tmem, b, h, qb);
+    cal_softmax<DPAD, QT>(tm, p, ctl, base, tmem, b, h, qb);
   }
   tc_fence_before();
   __syncthreads();

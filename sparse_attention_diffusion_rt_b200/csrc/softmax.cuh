@@ -65,6 +65,46 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BN], float s
   return lo + hi;
 }
 
+// As exp_pack_store, and also returns in xmax the largest x = s_c * sl2 - m of
+// the row block, so that a running max that is too small (x above the lazy
+// rescale threshold) is detected without a separate max pass: the max is taken
+// on the ALU pipe while the MUFU computes the exponentials.
+template <int BN>
+__device__ __forceinline__ float exp_pack_store_mx(const uint32_t (&s)[BN], float sl2, float m, uint32_t tP,
+                                                   float& xmax) {
+  uint64_t sum[4];
+  float mx[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sum[i] = 0ull;
+    mx[i] = -INFINITY;
+  }
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t neg_m2 = f2_pack(-m, -m);
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const uint64_t x = ffma2(f2_pack(__uint_as_float(s[c0 + 2 * c]), __uint_as_float(s[c0 + 2 * c + 1])),
+                               scale2, neg_m2);
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      mx[c & 3] = max3f(mx[c & 3], x0, x1);
+      const float p0 = ex2_approx(x0);
+      const float p1 = ex2_approx(x1);
+      sum[c & 3] = fadd2(sum[c & 3], f2_pack(p0, p1));
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_x32(tP + c0 / 2, pk);
+  }
+  xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  const uint64_t t = fadd2(fadd2(sum[0], sum[1]), fadd2(sum[2], sum[3]));
+  float lo, hi;
+  f2_unpack(t, lo, hi);
+  return lo + hi;
+}
+
 // Load BN fp32 logits of this thread's row from TMEM (caller waits with tmem_wait_ld).
 template <int BN>
 __device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[BN]) {
