@@ -179,6 +179,51 @@ def test_dense_and_empty_masks():
     assert torch.equal(o2, r_s)                # empty kept set: O' = R exactly
 
 
+@pytest.mark.parametrize("d", [72, 88, 128])
+@pytest.mark.parametrize("r_dtype", [torch.bfloat16, torch.float32])
+def test_dense_empty_and_mixed_rows_padded_dims(d, r_dtype):
+    """The d > 64 calibration keeps one accumulator and orders masked blocks
+    before kept ones: a row with no masked block, a row with no kept block and
+    rows with both take different paths through it."""
+    B, H, L, blk = 1, 2, 4 * 128 - 30, 128               # 4 query blocks, ragged tail
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=60 + d, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=160 + d, device=DEV)
+    mixed = np.array([[[1, 1, 1, 1],                      # dense row: no masked block
+                       [0, 0, 0, 0],                      # empty row: no kept block
+                       [0, 1, 0, 1],                      # kept blocks include the tail block
+                       [1, 0, 1, 0]]], dtype=np.uint8)    # the tail block is masked
+    _run_cycle_full(q, k, v, q2, k2, v2, mixed, blk, r_dtype=r_dtype)
+    o_full = ref.full_attention_ref(f64(q), f64(k), f64(v))
+    for mask, rho_want in ((np.ones((1, 4, 4), np.uint8), 1.0), (np.zeros((1, 4, 4), np.uint8), 0.0)):
+        o, rho, r = rt.rt_calibrate(q, k, v, _index(mask), block=blk, r_dtype=r_dtype)
+        torch.cuda.synchronize()
+        _ok()
+        assert torch.all(rho == rho_want)
+        check_out(f64(o), o_full, "calibrate O")
+        if rho_want == 1.0:
+            assert torch.all(r == 0)
+        else:
+            check_out(f64(r), o_full, "all-masked R is the full output")
+
+
+@pytest.mark.parametrize("vscale", [1e-3, 300.0])
+def test_residual_copy_row_scale_extremes(vscale):
+    """At d = 128 with a bf16 residual the masked-block accumulator is kept as
+    f16 with a power-of-two row scale; very small and very large V exercise
+    that scale.  Errors are compared in units of the V scale."""
+    B, H, L, d, blk = 1, 2, 3 * 128, 128, 128
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=71, device=DEV)
+    v = (v.float() * vscale).to(torch.bfloat16)
+    mask = np.array([[[1, 0, 0], [0, 1, 0], [1, 0, 1]]], dtype=np.uint8)
+    o, rho, r = rt.rt_calibrate(q, k, v, _index(mask), block=blk)
+    torch.cuda.synchronize()
+    _ok()
+    O, RHO, R = ref.calibrate_ref(f64(q), f64(k), f64(v), mask, blk)
+    check_out(f64(o) / vscale, O / vscale, "calibrate O / vscale")
+    check_out(f64(r) / vscale, R / vscale, "calibrate R / vscale")
+    check_rho(f64(rho), RHO)
+
+
 def test_invariant_same_inputs_lambda0_gives_full_attention():
     w = inputs.WORKLOADS["pixart"]
     q, k, v = inputs.initial_qkv(w, device=DEV)
