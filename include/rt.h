@@ -72,6 +72,24 @@ typedef enum rt_ramp {
 
 typedef enum rt_dtype { RT_BF16 = 0, RT_F32 = 1 } rt_dtype;
 
+/* What the calibration stores as the residual R (rt_calibrate_ex).
+ *   RT_RES_MASKED       Re-ttention's residual: the masked tokens' part of
+ *                       the full output, R_i = sum_{V(i)\M(i)} e^{s_ij-m_i} v_j / Z_full.
+ *   RT_RES_SUBTRACTIVE  DiTFastAttn's residual, the contrast the replies to W1
+ *                       work through: R_i = O_i - O_sparse_i with O_sparse_i the
+ *                       softmax over M(i) alone (0 when M(i) is empty). */
+typedef enum rt_residual { RT_RES_MASKED = 0, RT_RES_SUBTRACTIVE = 1 } rt_residual;
+
+/* Epilogue of the sparse step (rt_sparse_step_ex); attn_i is the softmax over
+ * M(i) of the step's own inputs (0 when M(i) is empty).
+ *   RT_EPI_RESHAPED  O'_i = ramp(rho_i, lambda, k) * attn_i + R_i   (Re-ttention)
+ *   RT_EPI_NO_RHO    O'_i = attn_i + R_i      (ablation without the statistical
+ *                    reshape; with an RT_RES_SUBTRACTIVE residual it is
+ *                    DiTFastAttn's reconstruction).  rho is not read (may be NULL).
+ *   RT_EPI_NO_R      O'_i = ramp(rho_i, lambda, k) * attn_i   (ablation without the
+ *                    residual).  r is not read (may be NULL). */
+typedef enum rt_epilogue { RT_EPI_RESHAPED = 0, RT_EPI_NO_RHO = 1, RT_EPI_NO_R = 2 } rt_epilogue;
+
 typedef struct rt_attn_desc {
   int32_t B, H, L, d;   /* batch, heads, tokens, head dimension */
   int32_t block;        /* query and key block size: 64 or 128 */
@@ -122,6 +140,23 @@ RT_API rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const voi
 RT_API rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                          const rt_block_index* idx, const float* rho, const void* r,
                          float lambda, int32_t step_distance, rt_ramp ramp, void* o, void* stream);
+
+/* rt_calibrate with the residual kind chosen: rt_calibrate(...) is
+ * rt_calibrate_ex(..., RT_RES_MASKED, stream).  Same arguments, layouts and
+ * errors; an unknown kind returns RT_ERR_INVALID_ARGUMENT. */
+RT_API rt_status rt_calibrate_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                          const rt_block_index* idx, void* o, float* rho, void* r, rt_residual kind,
+                          void* stream);
+
+/* rt_sparse_step with the epilogue chosen: rt_sparse_step(...) is
+ * rt_sparse_step_ex(..., RT_EPI_RESHAPED, o, stream).  rho may be NULL with
+ * RT_EPI_NO_RHO and r may be NULL with RT_EPI_NO_R (they are not read);
+ * otherwise as rt_sparse_step.  An unknown epilogue returns
+ * RT_ERR_INVALID_ARGUMENT. */
+RT_API rt_status rt_sparse_step_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                            const rt_block_index* idx, const float* rho, const void* r,
+                            float lambda, int32_t step_distance, rt_ramp ramp, rt_epilogue epi,
+                            void* o, void* stream);
 
 /* Synchronises `stream`, returns the first device-side status recorded since
  * the last call on the current device, and clears it. */

@@ -47,6 +47,11 @@ RAMP_MUL_LINEAR = 0
 RAMP_ADD_LINEAR = 1
 RAMP_GEOMETRIC = 2
 
+# sparse-step epilogues: Re-ttention's, and the two ablations the pages compare
+EPI_RESHAPED = 0      # rho_hat * attn + R
+EPI_NO_RHO = 1        # attn + R   (with R = O_full - O_sparse: DiTFastAttn's reconstruction)
+EPI_NO_R = 2          # rho_hat * attn
+
 
 # ---------------------------------------------------------------------------
 # masks
@@ -208,6 +213,27 @@ def ditfastattn_residual_ref(q, k, v, block_mask, block, scale=None):
     zero = np.zeros_like(q)
     o_sp = sparse_step_ref(q, k, v, block_mask, block, ones, zero, 0.0, 0, RAMP_MUL_LINEAR, scale)
     return o_full - o_sp
+
+
+def sparse_step_epilogue_ref(q, k, v, block_mask, block, rho, r, lam, kdist, epilogue=EPI_RESHAPED,
+                             mode=RAMP_MUL_LINEAR, scale=None):
+    """Sparse step with one of the epilogues the replies to W1 and the
+    ablation table set side by side.  attn is the softmax over the kept keys
+    (0 for a row with none):
+      EPI_RESHAPED  ramp(rho) * attn + R      (Re-ttention)
+      EPI_NO_RHO    attn + R                  (no statistical reshape; with
+                                               DiTFastAttn's R_sub this is its
+                                               reconstruction)
+      EPI_NO_R      ramp(rho) * attn          (no residual)
+    rho is not used by EPI_NO_RHO, r not by EPI_NO_R (either may be None)."""
+    B, H, L, d = q.shape
+    if epilogue == EPI_RESHAPED:
+        return sparse_step_ref(q, k, v, block_mask, block, rho, r, lam, kdist, mode, scale)
+    if epilogue == EPI_NO_RHO:
+        return sparse_step_ref(q, k, v, block_mask, block, np.ones((B, H, L)), r, 0.0, 0, mode, scale)
+    if epilogue == EPI_NO_R:
+        return sparse_step_ref(q, k, v, block_mask, block, rho, np.zeros_like(q), lam, kdist, mode, scale)
+    raise ValueError(f"unknown epilogue {epilogue}")
 
 
 def build_block_index_ref(block_mask):

@@ -67,6 +67,8 @@ struct AttnParams {
   float ramp_mul, ramp_add;
   float* rho_out;          // calibration
   int r_f32;
+  int use_rho, use_r;      // sparse-step epilogue: O' = (use_rho ? rho_hat : 1) * attn + (use_r ? R : 0)
+  int r_sub;               // calibration: R = O_full - O_sparse (subtractive residual) instead of the masked part
   unsigned long long wait_limit_ns;
   unsigned int* status;
 };
@@ -191,7 +193,9 @@ __device__ __forceinline__ void producer_role(const TmaSet& tm, const AttnParams
   const int q_row = qb * p.block;
   int issued = 0;
   bool ok = true;
-  if (!CAL) {
+  if (!CAL && !p.use_r) {
+    mbar_arrive(&ctl.r_full);               // no residual in this epilogue: nothing to load
+  } else if (!CAL) {
     // residual tile for the epilogue: independent of the main loop, issue first
     const uint32_t rbytes = p.r_f32 ? p.block * C::NCH32 * 128 : p.block * DPAD * 2;
     mbar_arrive_expect_tx(&ctl.r_full, rbytes);
@@ -432,13 +436,14 @@ __device__ __forceinline__ void softmax_role(const TmaSet& tm, const AttnParams&
   const bool row_ok = t < p.block;                   // rows of this query block (warp-uniform)
   const size_t rho_idx = (static_cast<size_t>(b) * p.H + h) * p.L + grow;
   if (ok && row_ok) {
-    float out_scale = 0.f;
+    float out_scale = 0.f, inv_in = 0.f;
     if (CAL) {
       out_scale = 1.f / (l + l_out);
+      inv_in = l > 0.f ? 1.f / l : 0.f;
       if (grow < p.L) p.rho_out[rho_idx] = l / (l + l_out);   // correctly rounded: dense mask gives 1
     } else {
-      const float rho = (grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
-      const float rho_hat = fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add));
+      const float rho = (p.use_rho && grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
+      const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
       out_scale = (n > 0) ? rho_hat / l : 0.f;
     }
 #pragma unroll
@@ -455,14 +460,20 @@ __device__ __forceinline__ void softmax_role(const TmaSet& tm, const AttnParams&
           const float xi = any_in ? __uint_as_float(ain[i]) : 0.f;
           const float xo = any_out ? __uint_as_float(aout[i]) : 0.f;
           a[i] = (xi + xo) * out_scale;
-          ro[i] = xo * out_scale;
+          // masked tokens' part, or O_full - O_sparse with O_sparse = acc_in / l_in (0 with no kept key)
+          ro[i] = p.r_sub ? a[i] - xi * inv_in : xo * out_scale;
         }
         store_row16<DPAD>(sStage, p.block, t, c, p.r_f32 != 0, ro);
       } else {
         uint32_t acc[16];
         if (n > 0) { tmem_ld_x16(tO + c, acc); tmem_wait_ld(); }
         float rr[16];
-        load_row16<DPAD>(sR, p.block, t, c, p.r_f32 != 0, rr);
+        if (p.use_r) {
+          load_row16<DPAD>(sR, p.block, t, c, p.r_f32 != 0, rr);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) a[i] = (n > 0 ? __uint_as_float(acc[i]) * out_scale : 0.f) + rr[i];
       }

@@ -334,6 +334,7 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     const float inv = 1.f / z;
     if (grow < p.L) p.rho_out[(static_cast<size_t>(b) * p.H + h) * p.L + grow] = l_in / z;
     const float rs = snap_scale * inv;
+    const float inv_in = l_in > 0.f ? 1.f / l_in : 0.f;
 #pragma unroll
     for (int c = 0; c < DPAD; c += 16) {
       uint32_t a[16], sv[16];
@@ -371,7 +372,8 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
           out_kept = 0.f;
         }
         o16[i] = out_masked + out_kept;
-        r16[i] = out_masked;
+        // masked tokens' part, or O_full - O_sparse with O_sparse = acc_in / l_in (0 with no kept key)
+        r16[i] = p.r_sub ? o16[i] - (n_masked < n ? acc * inv_in : 0.f) : out_masked;
       }
       store_row16<DPAD>(sO, 128, t, c, false, o16);
       store_row16<DPAD>(sRst, 128, t, c, p.r_f32 != 0, r16);

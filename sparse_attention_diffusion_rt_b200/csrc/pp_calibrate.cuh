@@ -223,6 +223,7 @@ __device__ __forceinline__ void pc_softmax(const TmaSet& tm, const AttnParams& p
   if (ok) {
     const float z = l_in + l_out;
     const float inv = 1.f / z;
+    const float inv_in = l_in > 0.f ? 1.f / l_in : 0.f;
     if (grow < p.L) p.rho_out[(static_cast<size_t>(b) * p.H + h) * p.L + grow] = l_in / z;
 #pragma unroll
     for (int h0 = 0; h0 < 64; h0 += 32) {
@@ -238,7 +239,8 @@ __device__ __forceinline__ void pc_softmax(const TmaSet& tm, const AttnParams& p
           const float xi = any_in ? __uint_as_float(ain[c + i]) : 0.f;
           const float xo = any_out ? __uint_as_float(aout[c + i]) : 0.f;
           o16[i] = (xi + xo) * inv;
-          r16[i] = xo * inv;
+          // masked tokens' part, or O_full - O_sparse with O_sparse = acc_in / l_in (0 with no kept key)
+          r16[i] = p.r_sub ? o16[i] - xi * inv_in : xo * inv;
         }
         store_row16<64>(sO, 128, t, h0 + c, false, o16);
         store_row16<64>(sRst, 128, t, h0 + c, p.r_f32 != 0, r16);

@@ -128,7 +128,7 @@ __device__ __forceinline__ void pp_producer(const TmaSet& tm, const AttnParams& 
       }
       if (!ok) break;
     }
-    if (!p.r_f32) {
+    if (!p.r_f32 && p.use_r) {
       if (ri >= 1 && !pp_wait(&P.r_empty, (ri - 1) & 1, ctl, p)) { ok = false; break; }
       mbar_arrive_expect_tx(&P.r_full, C::TILE);
       tma_load_4d(sR, &tm.r[0], &P.r_full, 0, q_row, h, b);
@@ -247,7 +247,7 @@ __device__ __forceinline__ void pp_softmax(const TmaSet& tm, const AttnParams& p
     if (ti.bad) continue;
     const int grow = ti.qb * 128 + t;
     const size_t rho_idx = (static_cast<size_t>(ti.b) * p.H + ti.h) * p.L + grow;
-    const float rho = grow < p.L ? __ldg(p.rho_in + rho_idx) : 0.f;
+    const float rho = (p.use_rho && grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
     float m = 0.f, l = 0.f;
     for (int j = 0; j < ti.n; ++j, ++g) {
       ok = __all_sync(0xffffffffu, pp_wait(&P.s_full, g & 1, ctl, p));
@@ -292,11 +292,11 @@ __device__ __forceinline__ void pp_softmax(const TmaSet& tm, const AttnParams& p
       tc_fence_after();
       ++oi;
     }
-    if (!p.r_f32) {
+    if (!p.r_f32 && p.use_r) {
       ok = __all_sync(0xffffffffu, pp_wait(&P.r_full, ri & 1, ctl, p));
       if (!ok) break;
     }
-    const float rho_hat = fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add));
+    const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
     const float scale = ti.n > 0 ? rho_hat / l : 0.f;
     // staging tile free once this thread's previous bulk store has read it
     if (t == 0) {
@@ -315,7 +315,10 @@ __device__ __forceinline__ void pp_softmax(const TmaSet& tm, const AttnParams& p
 #pragma unroll
       for (int c = h0; c < h0 + 32; c += 16) {
         float rr[16];
-        if (p.r_f32) {
+        if (!p.use_r) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+        } else if (p.r_f32) {
           if (grow < p.L) {
             const float4* src = reinterpret_cast<const float4*>(
                 static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
@@ -338,7 +341,7 @@ __device__ __forceinline__ void pp_softmax(const TmaSet& tm, const AttnParams& p
         store_row16<64>(sOst, 128, t, c, false, o16);
       }
     }
-    if (!p.r_f32) {
+    if (!p.r_f32 && p.use_r) {
       mbar_arrive(&P.r_empty);
       ++ri;
     }

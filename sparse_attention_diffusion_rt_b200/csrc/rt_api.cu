@@ -125,15 +125,19 @@ rt_status make_residual_maps(CUtensorMap (&m)[4], const void* ptr, const rt_attn
   return s;
 }
 
+// need_rho / need_r: whether the call reads (or writes) rho and R.
 rt_status validate(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
-                   const rt_block_index* idx, const void* o, const void* rho, const void* r) {
-  if (!desc || !idx || !q || !k || !v || !o || !rho || !r) return RT_ERR_INVALID_ARGUMENT;
+                   const rt_block_index* idx, const void* o, const void* rho, const void* r,
+                   bool need_rho = true, bool need_r = true) {
+  if (!desc || !idx || !q || !k || !v || !o) return RT_ERR_INVALID_ARGUMENT;
+  if ((need_rho && !rho) || (need_r && !r)) return RT_ERR_INVALID_ARGUMENT;
   const rt_attn_desc& d = *desc;
   if (d.B < 1 || d.H < 1 || d.L < 1 || d.d < 1) return RT_ERR_INVALID_ARGUMENT;
   if (d.stride_b < 1 || d.stride_h < 1 || d.stride_l < 1) return RT_ERR_INVALID_ARGUMENT;
   if (!(d.softmax_scale >= 0.f) || !std::isfinite(d.softmax_scale)) return RT_ERR_INVALID_ARGUMENT;
   if (d.r_dtype != RT_BF16 && d.r_dtype != RT_F32) return RT_ERR_INVALID_ARGUMENT;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(r) || !aligned16(rho))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (need_r && !aligned16(r)) ||
+      (need_rho && !aligned16(rho)))
     return RT_ERR_INVALID_ARGUMENT;
   if (d.d < 16 || d.d > 128 || d.d % 8 != 0) return RT_ERR_UNSUPPORTED;
   if (d.block != 64 && d.block != 128) return RT_ERR_UNSUPPORTED;
@@ -161,6 +165,9 @@ rt_status fill_common(const rt_attn_desc& d, const rt_block_index& idx, AttnPara
   const double c = d.softmax_scale > 0.f ? static_cast<double>(d.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d.d));
   p.scale_log2 = static_cast<float>(c * 1.4426950408889634);   // c * log2(e)
   p.r_f32 = d.r_dtype == RT_F32;
+  p.use_rho = 1;
+  p.use_r = 1;
+  p.r_sub = 0;
   p.wait_limit_ns = g_wait_limit_ns.load();
   return status_word(&p.status);
 }
@@ -243,6 +250,13 @@ rt_status rt_build_block_index(const uint8_t* d_mask, int32_t Hm, int32_t nqb, i
 
 rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                        const rt_block_index* idx, void* o, float* rho, void* r, void* stream) {
+  return rt_calibrate_ex(desc, q, k, v, idx, o, rho, r, RT_RES_MASKED, stream);
+}
+
+rt_status rt_calibrate_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                          const rt_block_index* idx, void* o, float* rho, void* r, rt_residual kind,
+                          void* stream) {
+  if (kind != RT_RES_MASKED && kind != RT_RES_SUBTRACTIVE) return RT_ERR_INVALID_ARGUMENT;
   rt_status st = validate(desc, q, k, v, idx, o, rho, r);
   if (st != RT_OK) return st;
   const rt_attn_desc& d = *desc;
@@ -250,6 +264,7 @@ rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const void* k, c
   AttnParams p;
   if ((st = fill_common(d, *idx, p)) != RT_OK) return st;
   p.rho_out = rho;
+  p.r_sub = kind == RT_RES_SUBTRACTIVE;
   TmaSet tm;
   std::memset(&tm, 0, sizeof(tm));
   if ((st = make_chunk_maps(tm.q, q, d, dpad, 128)) != RT_OK) return st;
@@ -264,7 +279,15 @@ rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const void* k, c
 rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                          const rt_block_index* idx, const float* rho, const void* r, float lambda,
                          int32_t step_distance, rt_ramp ramp, void* o, void* stream) {
-  rt_status st = validate(desc, q, k, v, idx, o, rho, r);
+  return rt_sparse_step_ex(desc, q, k, v, idx, rho, r, lambda, step_distance, ramp, RT_EPI_RESHAPED, o, stream);
+}
+
+rt_status rt_sparse_step_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
+                            const rt_block_index* idx, const float* rho, const void* r, float lambda,
+                            int32_t step_distance, rt_ramp ramp, rt_epilogue epi, void* o, void* stream) {
+  if (epi != RT_EPI_RESHAPED && epi != RT_EPI_NO_RHO && epi != RT_EPI_NO_R) return RT_ERR_INVALID_ARGUMENT;
+  const bool use_rho = epi != RT_EPI_NO_RHO, use_r = epi != RT_EPI_NO_R;
+  rt_status st = validate(desc, q, k, v, idx, o, rho, r, use_rho, use_r);
   if (st != RT_OK) return st;
   if (!std::isfinite(lambda) || step_distance < 0) return RT_ERR_INVALID_ARGUMENT;
   double mul = 1.0, add = 0.0;
@@ -279,8 +302,10 @@ rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k,
   const int dpad = dpad_of(d.d);
   AttnParams p;
   if ((st = fill_common(d, *idx, p)) != RT_OK) return st;
-  p.rho_in = rho;
-  p.r_in = r;
+  p.rho_in = use_rho ? rho : nullptr;
+  p.r_in = use_r ? r : nullptr;
+  p.use_rho = use_rho;
+  p.use_r = use_r;
   p.stride_b = d.stride_b;
   p.stride_h = d.stride_h;
   p.stride_l = d.stride_l;
@@ -292,7 +317,7 @@ rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k,
   if ((st = make_chunk_maps(tm.k, k, d, dpad, static_cast<uint32_t>(d.block))) != RT_OK) return st;
   if ((st = make_chunk_maps(tm.v, v, d, dpad, static_cast<uint32_t>(d.block))) != RT_OK) return st;
   if ((st = make_chunk_maps(tm.o, o, d, dpad, static_cast<uint32_t>(d.block))) != RT_OK) return st;
-  if ((st = make_residual_maps(tm.r, r, d, dpad)) != RT_OK) return st;
+  if (use_r && (st = make_residual_maps(tm.r, r, d, dpad)) != RT_OK) return st;
   cudaError_t e = dispatch(dpad, false, d, tm, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RT_OK : cuda_fail(e, "rt_sparse_step launch");
 }

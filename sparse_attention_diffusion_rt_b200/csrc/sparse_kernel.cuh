@@ -168,7 +168,7 @@ __device__ __forceinline__ void sp_producer(const TmaSet& tm, const AttnParams& 
         }
         if (!ok) break;
       }
-      if (!p.r_f32) {
+      if (!p.r_f32 && p.use_r) {
         if (ri >= 1 && !sp_wait(&ctl.r_empty, (ri - 1) & 1, ctl, p)) { ok = false; break; }
         mbar_arrive_expect_tx(&ctl.r_full, C::TILE_BYTES);
         tma_load_4d(sR, &tm.r[0], &ctl.r_full, 0, q_row, h, b);
@@ -307,7 +307,7 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
     if (ti.bad) continue;
     const int grow = ti.qb * 128 + t;
     const size_t rho_idx = (static_cast<size_t>(ti.b) * p.H + ti.h) * p.L + grow;
-    const float rho = grow < p.L ? __ldg(p.rho_in + rho_idx) : 0.f;
+    const float rho = (p.use_rho && grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
     float m = 0.f, l = 0.f;
     for (int j = 0; j < ti.n; ++j, ++g) {
       const int bf = g & 1;
@@ -353,11 +353,11 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       tc_fence_after();
       ++oi;
     }
-    if (!p.r_f32) {
+    if (!p.r_f32 && p.use_r) {
       ok = __all_sync(0xffffffffu, sp_wait(&ctl.r_full, ri & 1, ctl, p));
       if (!ok) break;
     }
-    const float rho_hat = fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add));
+    const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
     const float scale = ti.n > 0 ? rho_hat / l : 0.f;
     uint32_t packed[DPAD / 2];
 #pragma unroll
@@ -365,7 +365,10 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       uint32_t acc[16];
       if (ti.n > 0) { tmem_ld_x16(tO + c, acc); tmem_wait_ld(); }
       float rr[16];
-      if (p.r_f32) {
+      if (!p.use_r) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+      } else if (p.r_f32) {
         if (grow < p.L) {
           const float4* src = reinterpret_cast<const float4*>(
               static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
@@ -389,7 +392,7 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
         packed[c / 2 + i] = pack_bf16x2(a0, a1);
       }
     }
-    if (!p.r_f32) {
+    if (!p.r_f32 && p.use_r) {
       mbar_arrive(&ctl.r_empty);
       ++ri;
     }

@@ -35,10 +35,17 @@ RT_RAMP_GEOMETRIC = 2
 RT_BF16 = 0
 RT_F32 = 1
 
+RT_RES_MASKED = 0          # Re-ttention's residual (masked tokens' part of O)
+RT_RES_SUBTRACTIVE = 1     # DiTFastAttn's residual O - O_sparse
+
+RT_EPI_RESHAPED = 0        # O' = ramp(rho) * attn + R
+RT_EPI_NO_RHO = 1          # O' = attn + R
+RT_EPI_NO_R = 2            # O' = ramp(rho) * attn
+
 EXPORTED = (
-    "rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_check_device_error",
-    "rt_status_string", "rt_last_cuda_error", "rt_set_wait_limit_ns", "rt_debug_wait_timeout",
-    "rt_build_arch",
+    "rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
+    "rt_check_device_error", "rt_status_string", "rt_last_cuda_error", "rt_set_wait_limit_ns",
+    "rt_debug_wait_timeout", "rt_build_arch",
 )
 
 
@@ -86,6 +93,10 @@ def load_library() -> ctypes.CDLL:
                                  vp, vp, vp, vp]
     lib.rt_sparse_step.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
                                    vp, vp, ctypes.c_float, i32, ctypes.c_int, vp, vp]
+    lib.rt_calibrate_ex.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
+                                    vp, vp, vp, ctypes.c_int, vp]
+    lib.rt_sparse_step_ex.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
+                                      vp, vp, ctypes.c_float, i32, ctypes.c_int, ctypes.c_int, vp, vp]
     lib.rt_check_device_error.argtypes = [vp]
     lib.rt_status_string.argtypes = [ctypes.c_int]
     lib.rt_status_string.restype = ctypes.c_char_p
@@ -94,7 +105,8 @@ def load_library() -> ctypes.CDLL:
     lib.rt_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.rt_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.rt_build_arch.argtypes = []
-    for name in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_check_device_error",
+    for name in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
+                 "rt_check_device_error",
                  "rt_set_wait_limit_ns", "rt_debug_wait_timeout", "rt_build_arch"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -173,8 +185,10 @@ def _same_layout(ref: torch.Tensor, *ts):
 
 
 def rt_calibrate(q, k, v, index: BlockIndex, *, block: int, o=None, rho=None, r=None,
-                 r_dtype=torch.bfloat16, softmax_scale: float = 0.0, stream=None):
-    """Calibration step: returns (O bf16, rho fp32 [B,H,L], R r_dtype)."""
+                 r_dtype=torch.bfloat16, softmax_scale: float = 0.0, residual: int = RT_RES_MASKED,
+                 stream=None):
+    """Calibration step: returns (O bf16, rho fp32 [B,H,L], R r_dtype).
+    residual selects Re-ttention's R (default) or DiTFastAttn's O - O_sparse."""
     lib = load_library()
     _require_cuda(q, k, v, o, rho, r)
     for t in (q, k, v):
@@ -189,32 +203,41 @@ def rt_calibrate(q, k, v, index: BlockIndex, *, block: int, o=None, rho=None, r=
     _same_layout(q, k, v, o, r)
     desc = _desc(q, block, softmax_scale, r_dtype)
     idx = index.as_c()
-    _check(lib.rt_calibrate(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
-                            o.data_ptr(), rho.data_ptr(), r.data_ptr(), _stream_ptr(stream)),
+    _check(lib.rt_calibrate_ex(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
+                               o.data_ptr(), rho.data_ptr(), r.data_ptr(), int(residual), _stream_ptr(stream)),
            "rt_calibrate")
     return o, rho, r
 
 
 def rt_sparse_step(q, k, v, index: BlockIndex, rho, r, *, block: int, lam: float = 0.04,
                    step_distance: int = 1, ramp: int = RT_RAMP_MUL_LINEAR, o=None,
-                   softmax_scale: float = 0.0, stream=None):
-    """Reshaped sparse step: returns O' (bf16)."""
+                   softmax_scale: float = 0.0, epilogue: int = RT_EPI_RESHAPED, stream=None):
+    """Reshaped sparse step: returns O' (bf16).  epilogue selects the
+    Re-ttention epilogue (default) or an ablation; rho may be None with
+    RT_EPI_NO_RHO and r may be None with RT_EPI_NO_R."""
     lib = load_library()
     _require_cuda(q, k, v, rho, r, o)
     for t in (q, k, v):
         if t.dtype != torch.bfloat16:
             raise ValueError("q, k, v must be bfloat16")
-    if r.dtype not in (torch.bfloat16, torch.float32) or rho.dtype != torch.float32 or not rho.is_contiguous():
-        raise ValueError("r must be bf16/fp32, rho fp32 contiguous [B, H, L]")
+    if rho is None and epilogue != RT_EPI_NO_RHO:
+        raise ValueError("rho is required unless epilogue is RT_EPI_NO_RHO")
+    if r is None and epilogue != RT_EPI_NO_R:
+        raise ValueError("r is required unless epilogue is RT_EPI_NO_R")
+    if r is not None and r.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("r must be bf16 or fp32")
+    if rho is not None and (rho.dtype != torch.float32 or not rho.is_contiguous()):
+        raise ValueError("rho must be fp32 contiguous [B, H, L]")
     o = torch.empty_like(q) if o is None else o
     if o.dtype != torch.bfloat16:
         raise ValueError("o must be bfloat16")
-    _same_layout(q, k, v, o, r)
-    desc = _desc(q, block, softmax_scale, r.dtype)
+    _same_layout(q, k, v, o, *(() if r is None else (r,)))
+    desc = _desc(q, block, softmax_scale, torch.bfloat16 if r is None else r.dtype)
     idx = index.as_c()
-    _check(lib.rt_sparse_step(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
-                              rho.data_ptr(), r.data_ptr(), float(lam), int(step_distance), int(ramp),
-                              o.data_ptr(), _stream_ptr(stream)),
+    _check(lib.rt_sparse_step_ex(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
+                                 None if rho is None else rho.data_ptr(), None if r is None else r.data_ptr(),
+                                 float(lam), int(step_distance), int(ramp), int(epilogue),
+                                 o.data_ptr(), _stream_ptr(stream)),
            "rt_sparse_step")
     return o
 

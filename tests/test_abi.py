@@ -90,6 +90,22 @@ def test_host_validation_without_gpu(lib):
                               vp(4096), None) == rt.RT_ERR_INVALID_ARGUMENT     # unknown ramp
     assert lib.rt_sparse_step(ctypes.byref(desc), *args[:4], vp(4096), vp(4096), ctypes.c_float(0.04), -1, 0,
                               vp(4096), None) == rt.RT_ERR_INVALID_ARGUMENT     # negative step distance
+    # extended entry points: the residual kind and the epilogue are checked, and
+    # rho / r may be NULL only for the epilogue that does not read them
+    c_lam = ctypes.c_float(0.04)
+    assert lib.rt_calibrate_ex(ctypes.byref(desc), *args[:7], 5, None) == rt.RT_ERR_INVALID_ARGUMENT
+    sp = (ctypes.byref(desc), *args[:4])
+    assert lib.rt_sparse_step_ex(*sp, vp(4096), vp(4096), c_lam, 1, 0, 9, vp(4096), None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                           # unknown epilogue
+    for epi in (rt.RT_EPI_RESHAPED, rt.RT_EPI_NO_R):                         # these read rho
+        assert lib.rt_sparse_step_ex(*sp, None, vp(4096), c_lam, 1, 0, epi, vp(4096), None) == \
+            rt.RT_ERR_INVALID_ARGUMENT
+    for epi in (rt.RT_EPI_RESHAPED, rt.RT_EPI_NO_RHO):                       # these read r
+        assert lib.rt_sparse_step_ex(*sp, vp(4096), None, c_lam, 1, 0, epi, vp(4096), None) == \
+            rt.RT_ERR_INVALID_ARGUMENT
+    bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)
+    assert lib.rt_sparse_step_ex(ctypes.byref(bad), *args[:4], None, vp(4096), c_lam, 1, 0, rt.RT_EPI_NO_RHO,
+                                 vp(4096), None) == rt.RT_ERR_UNSUPPORTED   # NULL rho accepted, shape checked
     nnz = ctypes.c_int64(0)
     assert lib.rt_build_block_index(None, 1, 1, 1, vp(16), vp(16), 1, ctypes.byref(nnz), None) == \
         rt.RT_ERR_INVALID_ARGUMENT

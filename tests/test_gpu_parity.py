@@ -224,6 +224,48 @@ def test_residual_copy_row_scale_extremes(vscale):
     check_rho(f64(rho), RHO)
 
 
+@pytest.mark.parametrize("d,blk,r_dtype", [(64, 128, torch.bfloat16), (88, 128, torch.bfloat16),
+                                           (128, 128, torch.bfloat16), (128, 128, torch.float32),
+                                           (64, 64, torch.float32)])
+def test_epilogue_variants_and_subtractive_residual(d, blk, r_dtype):
+    """The ablation epilogues (no rho, no R) and DiTFastAttn's subtractive
+    residual with its reconstruction, on every kernel family (d = 64 ping-pong,
+    d > 64 persistent, 64-token blocks)."""
+    B, H, L = 1, 2, 3 * blk + 17
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=80 + d + blk, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=180 + d + blk, device=DEV)
+    nb = -(-L // blk)
+    mask = inputs.random_block_mask(1, nb, nb, 0.4, seed=81)
+    mask[0, 1, :] = 0                                   # one query block with no kept key block
+    idx = _index(mask)
+    lam, kd = 0.04, 2
+    # Re-ttention's residual, then the two ablations of the sparse step
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=blk, r_dtype=r_dtype)
+    o_norho = rt.rt_sparse_step(q2, k2, v2, idx, None, r, block=blk, lam=lam, step_distance=kd,
+                                epilogue=rt.RT_EPI_NO_RHO)
+    o_nor = rt.rt_sparse_step(q2, k2, v2, idx, rho, None, block=blk, lam=lam, step_distance=kd,
+                              epilogue=rt.RT_EPI_NO_R)
+    # DiTFastAttn: subtractive residual at calibration, attn + R_sub later
+    o_s, rho_s, r_sub = rt.rt_calibrate(q, k, v, idx, block=blk, r_dtype=r_dtype,
+                                        residual=rt.RT_RES_SUBTRACTIVE)
+    o_dfa = rt.rt_sparse_step(q2, k2, v2, idx, None, r_sub, block=blk, lam=lam, step_distance=kd,
+                              epilogue=rt.RT_EPI_NO_RHO)
+    torch.cuda.synchronize()
+    _ok()
+    O, RHO, R = ref.calibrate_ref(f64(q), f64(k), f64(v), mask, blk)
+    check_out(f64(o_s), O, "calibrate O (subtractive residual)")
+    check_rho(f64(rho_s), RHO)
+    R_SUB = ref.ditfastattn_residual_ref(f64(q), f64(k), f64(v), mask, blk)
+    check_out(f64(r_sub), R_SUB, "subtractive residual O - O_sparse")
+    args = (f64(q2), f64(k2), f64(v2), mask, blk)
+    check_out(f64(o_norho), ref.sparse_step_epilogue_ref(*args, None, f64(r), lam, kd, ref.EPI_NO_RHO),
+              "sparse O, no rho")
+    check_out(f64(o_nor), ref.sparse_step_epilogue_ref(*args, f64(rho), None, lam, kd, ref.EPI_NO_R),
+              "sparse O, no R")
+    check_out(f64(o_dfa), ref.sparse_step_epilogue_ref(*args, None, R_SUB, lam, kd, ref.EPI_NO_RHO),
+              "DiTFastAttn reconstruction")
+
+
 def test_invariant_same_inputs_lambda0_gives_full_attention():
     w = inputs.WORKLOADS["pixart"]
     q, k, v = inputs.initial_qkv(w, device=DEV)

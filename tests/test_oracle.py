@@ -86,6 +86,26 @@ def test_worked_example_ditfastattn_contrast():
     np.testing.assert_allclose(rec[0, 0, 0], g["step_t_plus_1"]["ditfastattn_reconstruction"], atol=1e-14)
 
 
+def test_worked_example_epilogue_variants():
+    """The named epilogues reproduce the worked example's rows: without R the
+    reshaped sparse row, without rho and with DiTFastAttn's R_sub its
+    reconstruction, and the full Re-ttention epilogue the full row."""
+    g = _worked_example()
+    mask = _window_mask(g["window_keys"])
+    q_t, k, v = _example_inputs(g["step_t"]["full"])
+    _, rho, r = ref.calibrate_ref(q_t, k, v, mask, 1)
+    r_sub = ref.ditfastattn_residual_ref(q_t, k, v, mask, 1)
+    q_t1, _, _ = _example_inputs(g["step_t_plus_1"]["full"])
+    no_r = ref.sparse_step_epilogue_ref(q_t1, k, v, mask, 1, rho, None, 0.0, 0, ref.EPI_NO_R)
+    np.testing.assert_allclose(no_r[0, 0, 0], g["step_t_plus_1"]["rettention_reshaped_sparse"], atol=1e-14)
+    no_rho = ref.sparse_step_epilogue_ref(q_t1, k, v, mask, 1, None, r_sub, 0.0, 0, ref.EPI_NO_RHO)
+    np.testing.assert_allclose(no_rho[0, 0, 0], g["step_t_plus_1"]["ditfastattn_reconstruction"], atol=1e-14)
+    full = ref.sparse_step_epilogue_ref(q_t1, k, v, mask, 1, rho, r, 0.0, 0, ref.EPI_RESHAPED)
+    np.testing.assert_allclose(full[0, 0, 0], g["step_t_plus_1"]["full"], atol=1e-14)
+    with pytest.raises(ValueError):
+        ref.sparse_step_epilogue_ref(q_t1, k, v, mask, 1, rho, r, 0.0, 0, 7)
+
+
 # ---------------------------------------------------------------------------
 # library routines and closed forms
 # ---------------------------------------------------------------------------
