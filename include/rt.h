@@ -158,6 +158,51 @@ RT_API rt_status rt_sparse_step_ex(const rt_attn_desc* desc, const void* q, cons
                             float lambda, int32_t step_distance, rt_ramp ramp, rt_epilogue epi,
                             void* o, void* stream);
 
+/* Denoising schedule: the pages calibrate (one full-attention step that
+ * refreshes the cached rho and R) every few denoising steps and run reshaped
+ * sparse steps in between, with the ramp-up growing with the distance to the
+ * calibration.  Step t = 0, 1, 2, ... of a schedule is a calibration when
+ * t % period == 0 and otherwise a sparse step at step distance
+ * k = t % period.  epilogue / residual select the method: Re-ttention is
+ * RT_EPI_RESHAPED + RT_RES_MASKED; DiTFastAttn's residual caching is
+ * RT_EPI_NO_RHO + RT_RES_SUBTRACTIVE. */
+typedef struct rt_schedule {
+  int32_t period;         /* calibration period T >= 1 */
+  float lambda;           /* ramp-up lambda of the sparse steps */
+  rt_ramp ramp;
+  rt_epilogue epilogue;
+  rt_residual residual;
+} rt_schedule;
+
+/* Step t of the schedule on this step's q, k, v: rt_calibrate_ex into o, rho
+ * and r at a calibration step, else rt_sparse_step_ex reading rho and r (the
+ * caller's cache, written by the last calibration step) into o.  Errors as
+ * those calls; t < 0, a NULL schedule or period < 1 return
+ * RT_ERR_INVALID_ARGUMENT. */
+RT_API rt_status rt_schedule_step(const rt_attn_desc* desc, const rt_schedule* sched, int32_t t,
+                           const void* q, const void* k, const void* v, const rt_block_index* idx,
+                           void* o, float* rho, void* r, void* stream);
+
+/* One whole calibration cycle (steps 0 .. period-1) captured as a CUDA graph,
+ * so that a cycle costs one launch.  q[t], k[t], v[t] and o[t] (arrays of
+ * `period` device pointers) are step t's buffers; rho and r the cache.  The
+ * graph reads and writes exactly those buffers every time it is launched.
+ * `stream` must be a created stream (capture is not possible on the legacy
+ * default stream: RT_ERR_INVALID_ARGUMENT).  Nothing is launched while
+ * capturing.  On success *graph receives a handle that the caller owns and
+ * releases with rt_cycle_graph_destroy. */
+typedef struct rt_cycle_graph rt_cycle_graph;
+RT_API rt_status rt_schedule_capture(const rt_attn_desc* desc, const rt_schedule* sched,
+                              const void* const* q, const void* const* k, const void* const* v,
+                              const rt_block_index* idx, void* const* o, float* rho, void* r,
+                              void* stream, rt_cycle_graph** graph);
+
+/* Launch a captured cycle on `stream` (asynchronous). */
+RT_API rt_status rt_cycle_graph_launch(rt_cycle_graph* graph, void* stream);
+
+/* Release a captured cycle (NULL is a no-op). */
+RT_API rt_status rt_cycle_graph_destroy(rt_cycle_graph* graph);
+
 /* Synchronises `stream`, returns the first device-side status recorded since
  * the last call on the current device, and clears it. */
 RT_API rt_status rt_check_device_error(void* stream);

@@ -52,6 +52,10 @@ EPI_RESHAPED = 0      # rho_hat * attn + R
 EPI_NO_RHO = 1        # attn + R   (with R = O_full - O_sparse: DiTFastAttn's reconstruction)
 EPI_NO_R = 2          # rho_hat * attn
 
+# residual kept by a calibration step
+RES_MASKED = 0        # Re-ttention: the masked tokens' part of the full output
+RES_SUBTRACTIVE = 1   # DiTFastAttn: O_full - O_sparse
+
 
 # ---------------------------------------------------------------------------
 # masks
@@ -234,6 +238,28 @@ def sparse_step_epilogue_ref(q, k, v, block_mask, block, rho, r, lam, kdist, epi
     if epilogue == EPI_NO_R:
         return sparse_step_ref(q, k, v, block_mask, block, rho, np.zeros_like(q), lam, kdist, mode, scale)
     raise ValueError(f"unknown epilogue {epilogue}")
+
+
+def schedule_ref(steps, block_mask, block, period, lam, mode=RAMP_MUL_LINEAR, epilogue=EPI_RESHAPED,
+                 residual=RES_MASKED, scale=None):
+    """Outputs of a denoising schedule: steps[t] = (q, k, v) of step t.  Step t
+    is a calibration (full attention; it refreshes the cached rho and
+    residual) when t % period == 0, else the sparse step at distance
+    t % period with the cached statistics, as the pages run Re-ttention
+    between periodic full-attention steps."""
+    outs = []
+    rho = r = None
+    for t, (q, k, v) in enumerate(steps):
+        kd = t % period
+        if kd == 0:
+            o, rho, r = calibrate_ref(q, k, v, block_mask, block, scale)
+            if residual == RES_SUBTRACTIVE:
+                r = ditfastattn_residual_ref(q, k, v, block_mask, block, scale)
+            outs.append(o)
+        else:
+            outs.append(sparse_step_epilogue_ref(q, k, v, block_mask, block, rho, r, lam, kd, epilogue, mode,
+                                                 scale))
+    return outs
 
 
 def build_block_index_ref(block_mask):

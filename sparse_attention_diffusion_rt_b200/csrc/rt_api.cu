@@ -20,6 +20,10 @@ cudaError_t launch_block_index(const uint8_t* mask, int rows, int nkb, int32_t* 
 
 using namespace rtb;
 
+namespace rtb {
+rt_status api_cuda_fail(cudaError_t e, const char* where);
+}
+
 namespace {
 
 // One status word per device (first device-side error since the last check).
@@ -52,6 +56,13 @@ rt_status status_word(unsigned int** out) {
   *out = cache[dev];
   return RT_OK;
 }
+
+}  // namespace
+
+// Records a CUDA error for rt_last_cuda_error (used by the other translation units).
+rt_status rtb::api_cuda_fail(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+
+namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -45,7 +45,8 @@ RT_EPI_NO_R = 2            # O' = ramp(rho) * attn
 EXPORTED = (
     "rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
     "rt_check_device_error", "rt_status_string", "rt_last_cuda_error", "rt_set_wait_limit_ns",
-    "rt_debug_wait_timeout", "rt_build_arch",
+    "rt_debug_wait_timeout", "rt_build_arch", "rt_schedule_step", "rt_schedule_capture",
+    "rt_cycle_graph_launch", "rt_cycle_graph_destroy",
 )
 
 
@@ -64,6 +65,11 @@ class RtBlockIndex(ctypes.Structure):
         ("nnz", ctypes.c_int64),
         ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
     ]
+
+
+class RtSchedule(ctypes.Structure):
+    _fields_ = [("period", ctypes.c_int32), ("lambda_", ctypes.c_float), ("ramp", ctypes.c_int),
+                ("epilogue", ctypes.c_int), ("residual", ctypes.c_int)]
 
 
 class RtError(RuntimeError):
@@ -97,6 +103,13 @@ def load_library() -> ctypes.CDLL:
                                     vp, vp, vp, ctypes.c_int, vp]
     lib.rt_sparse_step_ex.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, ctypes.POINTER(RtBlockIndex),
                                       vp, vp, ctypes.c_float, i32, ctypes.c_int, ctypes.c_int, vp, vp]
+    lib.rt_schedule_step.argtypes = [ctypes.POINTER(RtAttnDesc), ctypes.POINTER(RtSchedule), i32, vp, vp, vp,
+                                     ctypes.POINTER(RtBlockIndex), vp, vp, vp, vp]
+    vpp = ctypes.POINTER(vp)
+    lib.rt_schedule_capture.argtypes = [ctypes.POINTER(RtAttnDesc), ctypes.POINTER(RtSchedule), vpp, vpp, vpp,
+                                        ctypes.POINTER(RtBlockIndex), vpp, vp, vp, vp, ctypes.POINTER(vp)]
+    lib.rt_cycle_graph_launch.argtypes = [vp, vp]
+    lib.rt_cycle_graph_destroy.argtypes = [vp]
     lib.rt_check_device_error.argtypes = [vp]
     lib.rt_status_string.argtypes = [ctypes.c_int]
     lib.rt_status_string.restype = ctypes.c_char_p
@@ -106,6 +119,7 @@ def load_library() -> ctypes.CDLL:
     lib.rt_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.rt_build_arch.argtypes = []
     for name in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
+                 "rt_schedule_step", "rt_schedule_capture", "rt_cycle_graph_launch", "rt_cycle_graph_destroy",
                  "rt_check_device_error",
                  "rt_set_wait_limit_ns", "rt_debug_wait_timeout", "rt_build_arch"):
         getattr(lib, name).restype = ctypes.c_int
@@ -265,3 +279,73 @@ def rt_status_string(status: int) -> str:
 
 def rt_build_arch() -> int:
     return load_library().rt_build_arch()
+
+
+def _schedule(period, lam, ramp, epilogue, residual) -> RtSchedule:
+    return RtSchedule(int(period), float(lam), int(ramp), int(epilogue), int(residual))
+
+
+def rt_schedule_step(q, k, v, index: BlockIndex, t: int, *, block: int, period: int, o, rho, r,
+                     lam: float = 0.04, ramp: int = RT_RAMP_MUL_LINEAR, epilogue: int = RT_EPI_RESHAPED,
+                     residual: int = RT_RES_MASKED, softmax_scale: float = 0.0, stream=None):
+    """Step t of a denoising schedule: a calibration into (o, rho, r) when
+    t % period == 0, else a sparse step reading (rho, r) into o."""
+    lib = load_library()
+    _require_cuda(q, k, v, o, rho, r)
+    _same_layout(q, k, v, o, r)
+    desc = _desc(q, block, softmax_scale, r.dtype)
+    sched = _schedule(period, lam, ramp, epilogue, residual)
+    idx = index.as_c()
+    _check(lib.rt_schedule_step(ctypes.byref(desc), ctypes.byref(sched), int(t), q.data_ptr(), k.data_ptr(),
+                                v.data_ptr(), ctypes.byref(idx), o.data_ptr(), rho.data_ptr(), r.data_ptr(),
+                                _stream_ptr(stream)),
+           "rt_schedule_step")
+    return o
+
+
+class CycleGraph:
+    """One calibration cycle (steps 0 .. period-1) captured as a CUDA graph.
+    steps[t] = (q, k, v) and outs[t] = o of step t; rho and r are the cache.
+    The buffers must stay alive (and at the same addresses) while the graph
+    is used.  Capture needs a created stream (not the default stream)."""
+
+    def __init__(self, steps, index: BlockIndex, *, block: int, outs, rho, r, lam: float = 0.04,
+                 ramp: int = RT_RAMP_MUL_LINEAR, epilogue: int = RT_EPI_RESHAPED, residual: int = RT_RES_MASKED,
+                 softmax_scale: float = 0.0, stream: torch.cuda.Stream):
+        lib = load_library()
+        period = len(steps)
+        if period < 1 or len(outs) != period:
+            raise ValueError("one (q, k, v) and one output per step of the cycle")
+        for (q, k, v), o in zip(steps, outs):
+            _require_cuda(q, k, v, o)
+            _same_layout(steps[0][0], q, k, v, o, r)
+        _require_cuda(rho, r)
+        if stream is None or stream.cuda_stream == 0:
+            raise ValueError("capture needs a created stream")
+        desc = _desc(steps[0][0], block, softmax_scale, r.dtype)
+        sched = _schedule(period, lam, ramp, epilogue, residual)
+        arr = lambda xs: (ctypes.c_void_p * period)(*[x.data_ptr() for x in xs])
+        self._keep = (steps, outs, rho, r, index)       # keep the captured buffers alive
+        idx = index.as_c()
+        h = ctypes.c_void_p()
+        _check(lib.rt_schedule_capture(ctypes.byref(desc), ctypes.byref(sched), arr([s[0] for s in steps]),
+                                       arr([s[1] for s in steps]), arr([s[2] for s in steps]), ctypes.byref(idx),
+                                       arr(outs), rho.data_ptr(), r.data_ptr(), ctypes.c_void_p(stream.cuda_stream),
+                                       ctypes.byref(h)),
+               "rt_schedule_capture")
+        self._h = h
+        self.period = period
+
+    def launch(self, stream=None):
+        _check(load_library().rt_cycle_graph_launch(self._h, _stream_ptr(stream)), "rt_cycle_graph_launch")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _check(load_library().rt_cycle_graph_destroy(self._h), "rt_cycle_graph_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

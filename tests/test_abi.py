@@ -56,15 +56,18 @@ def test_struct_layout_matches_c(tmp_path):
     src = tmp_path / "layout.c"
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "rt.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(rt_attn_desc),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(rt_attn_desc),"
         " offsetof(rt_attn_desc, stride_b), offsetof(rt_attn_desc, softmax_scale), offsetof(rt_attn_desc, r_dtype),"
-        " sizeof(rt_block_index), offsetof(rt_block_index, nnz), offsetof(rt_block_index, col_idx));return 0;}\n")
+        " sizeof(rt_block_index), offsetof(rt_block_index, nnz), offsetof(rt_block_index, col_idx),"
+        " sizeof(rt_schedule), offsetof(rt_schedule, lambda), offsetof(rt_schedule, epilogue),"
+        " offsetof(rt_schedule, residual));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
     got = list(map(int, subprocess.check_output([str(exe)]).split()))
     want = [ctypes.sizeof(rt.RtAttnDesc), rt.RtAttnDesc.stride_b.offset, rt.RtAttnDesc.softmax_scale.offset,
             rt.RtAttnDesc.r_dtype.offset, ctypes.sizeof(rt.RtBlockIndex), rt.RtBlockIndex.nnz.offset,
-            rt.RtBlockIndex.col_idx.offset]
+            rt.RtBlockIndex.col_idx.offset, ctypes.sizeof(rt.RtSchedule), rt.RtSchedule.lambda_.offset,
+            rt.RtSchedule.epilogue.offset, rt.RtSchedule.residual.offset]
     assert got == want
 
 
@@ -106,6 +109,22 @@ def test_host_validation_without_gpu(lib):
     bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)
     assert lib.rt_sparse_step_ex(ctypes.byref(bad), *args[:4], None, vp(4096), c_lam, 1, 0, rt.RT_EPI_NO_RHO,
                                  vp(4096), None) == rt.RT_ERR_UNSUPPORTED   # NULL rho accepted, shape checked
+    # schedule driver: the schedule and t are checked before any CUDA call
+    sched = rt.RtSchedule(5, 0.04, 0, 0, 0)
+    cal_args = (vp(4096), vp(4096), vp(4096), ctypes.byref(idx), vp(4096), vp(4096), vp(4096), None)
+    assert lib.rt_schedule_step(ctypes.byref(desc), None, 0, *cal_args) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_schedule_step(ctypes.byref(desc), ctypes.byref(sched), -1, *cal_args) == rt.RT_ERR_INVALID_ARGUMENT
+    zero = rt.RtSchedule(0, 0.04, 0, 0, 0)
+    assert lib.rt_schedule_step(ctypes.byref(desc), ctypes.byref(zero), 3, *cal_args) == rt.RT_ERR_INVALID_ARGUMENT
+    bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)
+    assert lib.rt_schedule_step(ctypes.byref(bad), ctypes.byref(sched), 0, *cal_args) == rt.RT_ERR_UNSUPPORTED
+    assert lib.rt_schedule_step(ctypes.byref(bad), ctypes.byref(sched), 2, *cal_args) == rt.RT_ERR_UNSUPPORTED
+    h = ctypes.c_void_p(1)
+    assert lib.rt_schedule_capture(ctypes.byref(desc), ctypes.byref(sched), None, None, None, ctypes.byref(idx),
+                                   None, vp(4096), vp(4096), None, ctypes.byref(h)) == rt.RT_ERR_INVALID_ARGUMENT
+    assert h.value is None                                                   # the handle is cleared on error
+    assert lib.rt_cycle_graph_launch(None, None) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_cycle_graph_destroy(None) == rt.RT_OK
     nnz = ctypes.c_int64(0)
     assert lib.rt_build_block_index(None, 1, 1, 1, vp(16), vp(16), 1, ctypes.byref(nnz), None) == \
         rt.RT_ERR_INVALID_ARGUMENT

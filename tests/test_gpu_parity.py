@@ -266,6 +266,77 @@ def test_epilogue_variants_and_subtractive_residual(d, blk, r_dtype):
               "DiTFastAttn reconstruction")
 
 
+def _drifting_steps(B, H, L, d, n, seed):
+    x = inputs.random_qkv(B, H, L, d, seed=seed, device=DEV)
+    steps = [x]
+    g = torch.Generator(device=DEV).manual_seed(seed + 1)
+    for _ in range(n - 1):
+        x = tuple((t.float() + 0.05 * torch.randn(t.shape, generator=g, device=DEV)).to(torch.bfloat16)
+                  for t in x)
+        steps.append(x)
+    return steps
+
+
+@pytest.mark.parametrize("d,epilogue,residual", [(64, rt.RT_EPI_RESHAPED, rt.RT_RES_MASKED),
+                                                 (128, rt.RT_EPI_RESHAPED, rt.RT_RES_MASKED),
+                                                 (88, rt.RT_EPI_NO_RHO, rt.RT_RES_SUBTRACTIVE)])
+def test_schedule_steps_match_oracle_schedule(d, epilogue, residual):
+    """Seven denoising steps with a calibration every three, on inputs that
+    drift from step to step: Re-ttention's schedule and DiTFastAttn's."""
+    B, H, L, blk, period, lam = 1, 2, 3 * 128 - 40, 128, 3, 0.04
+    steps = _drifting_steps(B, H, L, d, 7, seed=90 + d)
+    mask = inputs.random_block_mask(1, 3, 3, 0.5, seed=91, ensure_nonempty=True)
+    idx = _index(mask)
+    rho = torch.empty((B, H, L), dtype=torch.float32, device=DEV)
+    r = torch.empty_like(steps[0][0])
+    outs = []
+    for t, (q, k, v) in enumerate(steps):
+        outs.append(rt.rt_schedule_step(q, k, v, idx, t, block=blk, period=period, lam=lam, o=torch.empty_like(q),
+                                        rho=rho, r=r, epilogue=epilogue, residual=residual))
+    torch.cuda.synchronize()
+    _ok()
+    want = ref.schedule_ref([tuple(f64(x) for x in s) for s in steps], mask, blk, period, lam,
+                            epilogue=epilogue, residual=residual)
+    for t, (o, w) in enumerate(zip(outs, want)):
+        check_out(f64(o), w, f"schedule step {t}")
+
+
+def test_cycle_graph_replays_the_eager_cycle_bit_exactly():
+    """A captured calibration cycle launched twice gives exactly the outputs of
+    the same steps run one call at a time (one launch per cycle instead of
+    `period`)."""
+    B, H, L, d, blk, period = 1, 2, 4 * 128, 128, 128, 4
+    steps = _drifting_steps(B, H, L, d, period, seed=95)
+    mask = inputs.random_block_mask(1, 4, 4, 0.4, seed=96, ensure_nonempty=True)
+    idx = _index(mask)
+    rho = torch.empty((B, H, L), dtype=torch.float32, device=DEV)
+    r = torch.empty_like(steps[0][0])
+    eager = [rt.rt_schedule_step(q, k, v, idx, t, block=blk, period=period, o=torch.empty_like(q), rho=rho, r=r)
+             for t, (q, k, v) in enumerate(steps)]
+    torch.cuda.synchronize()
+    _ok()
+    eager = [o.clone() for o in eager]
+    outs = [torch.zeros_like(steps[0][0]) for _ in range(period)]
+    rho_g, r_g = torch.empty_like(rho), torch.empty_like(r)
+    s = torch.cuda.Stream()
+    graph = rt.CycleGraph(steps, idx, block=blk, outs=outs, rho=rho_g, r=r_g, stream=s)
+    try:
+        torch.cuda.synchronize()
+        assert all(torch.count_nonzero(o) == 0 for o in outs)      # capturing launched nothing
+        for _ in range(2):
+            graph.launch(stream=s)
+            s.synchronize()
+            _ok()
+            for o, e in zip(outs, eager):
+                assert torch.equal(o, e)
+            assert torch.equal(rho_g, rho) and torch.equal(r_g, r)
+            for o in outs:
+                o.zero_()
+            torch.cuda.synchronize()                              # zeroed before the next replay writes
+    finally:
+        graph.close()
+
+
 def test_invariant_same_inputs_lambda0_gives_full_attention():
     w = inputs.WORKLOADS["pixart"]
     q, k, v = inputs.initial_qkv(w, device=DEV)

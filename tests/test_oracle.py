@@ -106,6 +106,40 @@ def test_worked_example_epilogue_variants():
         ref.sparse_step_epilogue_ref(q_t1, k, v, mask, 1, rho, r, 0.0, 0, 7)
 
 
+def test_worked_example_as_a_schedule():
+    """The worked example is a two-step schedule: a calibration at t, then the
+    step t+1 from the cached statistics.  Re-ttention reconstructs the full row
+    exactly; DiTFastAttn's residual caching gives its printed row."""
+    g = _worked_example()
+    mask = _window_mask(g["window_keys"])
+    q_t, k, v = _example_inputs(g["step_t"]["full"])
+    q_t1, _, _ = _example_inputs(g["step_t_plus_1"]["full"])
+    steps = [(q_t, k, v), (q_t1, k, v)]
+    outs = ref.schedule_ref(steps, mask, 1, 2, 0.0)
+    np.testing.assert_allclose(outs[0][0, 0, 0], g["step_t"]["full"], atol=1e-14)
+    np.testing.assert_allclose(outs[1][0, 0, 0], g["step_t_plus_1"]["rettention_reconstruction"], atol=1e-14)
+    dfa = ref.schedule_ref(steps, mask, 1, 2, 0.0, epilogue=ref.EPI_NO_RHO, residual=ref.RES_SUBTRACTIVE)
+    np.testing.assert_allclose(dfa[1][0, 0, 0], g["step_t_plus_1"]["ditfastattn_reconstruction"], atol=1e-14)
+
+
+def test_schedule_period_one_is_full_attention_and_static_inputs_stay_exact():
+    q, k, v = (_rand((1, 2, 96, 8), s) for s in (1, 2, 3))
+    q2 = q + 0.1 * _rand(q.shape, 4)
+    mask = np.array([[[1, 0, 0], [0, 1, 1], [1, 0, 1]]], dtype=np.uint8)
+    full = [ref.full_attention_ref(*x) for x in ((q, k, v), (q2, k, v))]
+    outs = ref.schedule_ref([(q, k, v), (q2, k, v)], mask, 32, 1, 0.04)       # every step calibrates
+    for o, f in zip(outs, full):
+        np.testing.assert_allclose(o, f, atol=1e-12)
+    # unchanged inputs and no ramp: every sparse step reproduces full attention
+    outs = ref.schedule_ref([(q, k, v)] * 4, mask, 32, 4, 0.0)
+    for o in outs:
+        np.testing.assert_allclose(o, full[0], atol=1e-12)
+    # with a ramp the sparse steps move away from it, more with the step distance
+    outs = ref.schedule_ref([(q, k, v)] * 4, mask, 32, 4, 0.04)
+    errs = [np.abs(o - full[0]).max() for o in outs]
+    assert errs[0] < 1e-12 and 0 < errs[1] < errs[2] < errs[3]
+
+
 # ---------------------------------------------------------------------------
 # library routines and closed forms
 # ---------------------------------------------------------------------------
