@@ -17,7 +17,9 @@ Metric: executed-block TFLOP/s (4 * block^2 * d * kept blocks * B * H per
 attention call, true d; calibration executes every block).  The line also
 carries per-kernel latency/TFLOP/s, the roofline object of the dominant
 kernel, the CPU oracle baseline, the end-to-end number through the public API
-with host buffers, and the SM clocks seen during the timed region.
+with host buffers, one denoising-schedule cycle (call by call and as a captured
+CUDA graph, with each step's error against full attention), and the SM clocks
+seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 Multi-GPU (weak scaling, independent replicas, no data-path collective):
@@ -239,6 +241,72 @@ def cpu_oracle_sample(w, qkv_steps_cpu, mask, budget_s=15.0):
     return flops / dt / 1e12, desc, cores
 
 
+def measure_schedule(w, mask, rt, period=5, reps=3):
+    """One calibration cycle of the denoising-schedule driver on drifting inputs:
+    the cycle run call by call and as one captured CUDA graph (device time per
+    cycle), and each step's relative L2 error against full attention on that
+    step's inputs, for Re-ttention, the no-rho ablation and DiTFastAttn."""
+    dev = mask.device
+    steps = inputs.qkv_steps(w, period, device=dev)
+    idx = rt.rt_build_block_index(mask)
+    q0 = steps[0][0]
+    rho = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    r = torch.empty_like(q0)
+    outs = [torch.empty_like(q0) for _ in range(period)]
+    s = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def eager(epilogue=rt.RT_EPI_RESHAPED, residual=rt.RT_RES_MASKED):
+        for t, (q, k, v) in enumerate(steps):
+            rt.rt_schedule_step(q, k, v, idx, t, block=w.block, period=period, lam=w.lam, o=outs[t], rho=rho,
+                                r=r, epilogue=epilogue, residual=residual, stream=s)
+
+    with torch.cuda.stream(s):
+        eager()
+        s.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record(s)
+        for _ in range(reps):
+            eager()
+        e1.record(s)
+        s.synchronize()
+        eager_ms = e0.elapsed_time(e1) / reps
+    graph = rt.CycleGraph(steps, idx, block=w.block, outs=outs, rho=rho, r=r, lam=w.lam, stream=s)
+    try:
+        graph.launch(stream=s)
+        s.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record(s)
+        for _ in range(reps):
+            graph.launch(stream=s)
+        e1.record(s)
+        s.synchronize()
+        graph_ms = e0.elapsed_time(e1) / reps
+    finally:
+        graph.close()
+    # full attention of every step (the calibration kernel's O), then each method's outputs
+    full = []
+    for q, k, v in steps:
+        o_full, _, _ = rt.rt_calibrate(q, k, v, idx, block=w.block)
+        full.append(o_full.float())
+    errs = {}
+    for name, epi, res in (("rettention", rt.RT_EPI_RESHAPED, rt.RT_RES_MASKED),
+                           ("no_rho", rt.RT_EPI_NO_RHO, rt.RT_RES_MASKED),
+                           ("ditfastattn", rt.RT_EPI_NO_RHO, rt.RT_RES_SUBTRACTIVE)):
+        with torch.cuda.stream(s):
+            eager(epi, res)
+        s.synchronize()
+        errs[name] = [float(torch.linalg.vector_norm(o.float() - f) / torch.linalg.vector_norm(f))
+                      for o, f in zip(outs, full)]
+    st = rt.rt_check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the schedule run: {rt.rt_status_string(st)}")
+    return {"period": period, "cycle": f"1 calibration + {period - 1} sparse steps (k = 1..{period - 1})",
+            "cycle_ms_call_by_call": eager_ms, "cycle_ms_graph": graph_ms, "launches_per_cycle_graph": 1,
+            "rel_l2_err_vs_full_per_step": errs,
+            "inputs": "synthetic, each step adds 0.05*N(0,1) to Q/K/V (errors are of the synthetic drift)"}
+
+
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
@@ -452,6 +520,13 @@ def run_ours(args, rank, world, local_rank):
     except Exception as exc:  # noqa: BLE001
         sdpa = {"error": str(exc)[:200]}
 
+    schedule = None
+    if not args.no_schedule:
+        try:
+            schedule = measure_schedule(w, mask, rt)
+        except torch.cuda.OutOfMemoryError as exc:
+            schedule = {"error": str(exc)[:200]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         steps_cpu = [tuple(x[:, :1].cpu() for x in qkv[0]), tuple(x[:, :1].cpu() for x in qkv[1])]
@@ -476,6 +551,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline_sparse_step": roof("sparse_step", sp_ms, sp_flops, sp_tf),
             "cpu_baseline": cpu,
             "context_torch_sdpa": sdpa,
+            "schedule": schedule,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
@@ -492,6 +568,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-schedule", action="store_true",
+                    help="skip the denoising-schedule driver measurement (one captured cycle)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (a smaller case for profiling)")
