@@ -18,8 +18,9 @@ attention call, true d; calibration executes every block).  The line also
 carries per-kernel latency/TFLOP/s, the roofline object of the dominant
 kernel, the CPU oracle baseline, the end-to-end number through the public API
 with host buffers, one denoising-schedule cycle (call by call and as a captured
-CUDA graph, with each step's error against full attention), and the SM clocks
-seen during the timed region.
+CUDA graph, with each step's error against full attention), the token
+reordering (the permutation's bandwidth and the mask's locality on raster vs
+Hilbert-ordered tokens), and the SM clocks seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 Multi-GPU (weak scaling, independent replicas, no data-path collective):
@@ -239,6 +240,76 @@ def cpu_oracle_sample(w, qkv_steps_cpu, mask, budget_s=15.0):
             f"({n_cal}/{w.B * w.H * nqb} of the cycle's calibration units) in {dt:.1f} s; "
             f"executed-block FLOPs of the sample / CPU time")
     return flops / dt / 1e12, desc, cores
+
+
+def mask_locality(w, mask, perm=None):
+    """How local a static block mask is on the latent grid: the fraction of
+    each visual token's 26 grid neighbours that lie in the key blocks kept for
+    its query block (neighbour recall), and the mean bounding-box volume, in
+    grid cells, of the visual tokens of a block."""
+    coords = inputs.token_coords(w, perm)
+    F, Y, X = w.grid
+    raster = np.arange(w.L) if perm is None else np.asarray(perm, dtype=np.int64)
+    pos = np.empty(w.L, dtype=np.int64)
+    pos[raster] = np.arange(w.L)                      # raster index -> position
+    vis = np.nonzero(~np.isnan(coords[:, 0]))[0]
+    c = coords[vis].astype(np.int64)
+    m = mask[0].astype(bool)
+    hit = total = 0
+    for df in (-1, 0, 1):
+        for dy in (-1, 0, 1):
+            for dx in (-1, 0, 1):
+                if df == dy == dx == 0:
+                    continue
+                nb = c + np.array([df, dy, dx])
+                ok = ((nb >= 0) & (nb < np.array([F, Y, X]))).all(axis=1)
+                j = pos[w.n_text + (nb[ok, 0] * Y + nb[ok, 1]) * X + nb[ok, 2]]
+                hit += int(m[vis[ok] // w.block, j // w.block].sum())
+                total += int(ok.sum())
+    blk = vis // w.block
+    vols = []
+    for b in np.unique(blk):
+        cb = c[blk == b]
+        vols.append(float(np.prod(cb.max(axis=0) - cb.min(axis=0) + 1)))
+    return hit / max(total, 1), float(np.mean(vols))
+
+
+def measure_token_order(w, rt, reps=5):
+    """The reordering row: the Hilbert token order, the device permutation's
+    bandwidth on one [B, H, L, d] tensor (read + write), and the mask's
+    locality on raster vs reordered tokens at the same kept blocks per row."""
+    if w.grid is None:
+        return None
+    perm_h = rt.rt_hilbert_token_order(w.n_text, *w.grid)
+    perm = perm_h.cuda()
+    x = inputs.initial_qkv(w, device="cuda")[0]
+    y = torch.empty_like(x)
+    for _ in range(2):
+        rt.rt_permute_tokens(x, perm, dst=y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        rt.rt_permute_tokens(x, perm, dst=y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = 2 * x.numel() * x.element_size()
+    ok = bool(torch.equal(y, x[:, :, perm.long()]))
+    st = rt.rt_check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the permutation: {rt.rt_status_string(st)}")
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    rec_r, vol_r = mask_locality(w, inputs.block_mask(w))
+    rec_h, vol_h = mask_locality(w, inputs.block_mask(w, perm_h.numpy()), perm_h.numpy())
+    return {"order": "text first, then the grid along its Hilbert curve",
+            "permute_ms": ms, "permute_bytes": nbytes, "permute_gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"]},
+            "permute_matches_torch_indexing": ok, "kept_blocks_per_row": w.kept,
+            "neighbour_recall": {"raster": rec_r, "hilbert": rec_h},
+            "block_bbox_cells": {"raster": vol_r, "hilbert": vol_h}}
 
 
 def measure_schedule(w, mask, rt, period=5, reps=3):
@@ -527,6 +598,10 @@ def run_ours(args, rank, world, local_rank):
         except torch.cuda.OutOfMemoryError as exc:
             schedule = {"error": str(exc)[:200]}
 
+    token_order = None
+    if not args.no_schedule:
+        token_order = measure_token_order(w, rt)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         steps_cpu = [tuple(x[:, :1].cpu() for x in qkv[0]), tuple(x[:, :1].cpu() for x in qkv[1])]
@@ -552,6 +627,7 @@ def run_ours(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "context_torch_sdpa": sdpa,
             "schedule": schedule,
+            "token_order": token_order,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
@@ -569,7 +645,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-schedule", action="store_true",
-                    help="skip the denoising-schedule driver measurement (one captured cycle)")
+                    help="skip the denoising-schedule and token-order measurements")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (a smaller case for profiling)")

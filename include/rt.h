@@ -203,6 +203,31 @@ RT_API rt_status rt_cycle_graph_launch(rt_cycle_graph* graph, void* stream);
 /* Release a captured cycle (NULL is a no-op). */
 RT_API rt_status rt_cycle_graph_destroy(rt_cycle_graph* graph);
 
+/* Token order that makes the blocks of the static mask compact (the pages
+ * lay video tokens out along a space-filling curve before blocking them).
+ * Tokens in raster order are n_text text tokens, then an F x Y x X latent
+ * grid with x fastest.  h_perm (host, n_text + F*Y*X entries) receives, for
+ * each position i of the new order, the raster index of the token placed
+ * there: the text tokens stay first, and the grid follows the Hilbert curve
+ * (over the axes longer than 1) of the smallest enclosing cube of side 2^b,
+ * restricted to the grid.
+ * 128 consecutive tokens then fill a compact brick instead of a row strip.
+ * Attention and every per-token operation commute with a fixed permutation,
+ * so a model applies it once where tokens are formed (rt_permute_tokens) and
+ * builds the block mask on the reordered tokens. */
+RT_API rt_status rt_hilbert_token_order(int32_t n_text, int32_t F, int32_t Y, int32_t X, int32_t* h_perm);
+
+/* Reorder the token rows of a bf16 [B, H, L, d] tensor (layout and strides of
+ * `desc`; B, H, L, d and the strides are used, the rest ignored):
+ *   inverse = 0: dst[b, h, i, :] = src[b, h, perm[i], :]   (raster -> new order)
+ *   inverse = 1: dst[b, h, perm[i], :] = src[b, h, i, :]   (back to raster order)
+ * d_perm: device i32 [L], a permutation of 0..L-1.  An entry outside [0, L)
+ * records RT_ERR_BAD_INDEX in the device status word and its row is skipped.
+ * src and dst must not overlap.  d % 8 == 0, 16-byte aligned pointers and
+ * strides that are multiples of 8 elements.  Asynchronous on `stream`. */
+RT_API rt_status rt_permute_tokens(const rt_attn_desc* desc, const void* src, void* dst, const int32_t* d_perm,
+                            int32_t inverse, void* stream);
+
 /* Synchronises `stream`, returns the first device-side status recorded since
  * the last call on the current device, and clears it. */
 RT_API rt_status rt_check_device_error(void* stream);

@@ -262,6 +262,63 @@ def schedule_ref(steps, block_mask, block, period, lam, mode=RAMP_MUL_LINEAR, ep
     return outs
 
 
+def hilbert_order_ref(n_text, F, Y, X):
+    """Token order of the reordering row: text tokens first (unchanged), then
+    the F x Y x X grid (raster index n_text + (f*Y + y)*X + x) sorted by the
+    Hilbert index, over the axes longer than 1, within the smallest cube of
+    side 2^b that holds the grid.  The index follows Skilling's transpose
+    method ("Programming the Hilbert curve", 2004), evaluated here for all
+    grid points at once.  Returns perm (int64 [L]): position i holds raster
+    token perm[i]."""
+    ext = [F, Y, X]
+    bits = 0
+    while (1 << bits) < max(ext):
+        bits += 1
+    f, y, x = np.meshgrid(np.arange(F), np.arange(Y), np.arange(X), indexing="ij")
+    axes = [c.ravel().astype(np.int64) for c, e in zip((f, y, x), ext) if e > 1]
+    n = len(axes)
+    if n == 0:
+        return np.arange(n_text + 1)
+    a = [c.copy() for c in axes]
+    q = 1 << (bits - 1) if bits > 0 else 0
+    while q > 1:
+        low = q - 1
+        for i in range(n):
+            hit = (a[i] & q) != 0
+            swap = (a[0] ^ a[i]) & low
+            a0_new = np.where(hit, a[0] ^ low, a[0] ^ swap)
+            ai_new = np.where(hit, a[i], a[i] ^ swap) if i > 0 else a0_new
+            a[0] = a0_new
+            if i > 0:
+                a[i] = ai_new
+        q >>= 1
+    for i in range(1, n):
+        a[i] = a[i] ^ a[i - 1]
+    t = np.zeros_like(a[0])
+    q = 1 << (bits - 1) if bits > 0 else 0
+    while q > 1:
+        t = np.where((a[n - 1] & q) != 0, t ^ (q - 1), t)
+        q >>= 1
+    a = [c ^ t for c in a]
+    key = np.zeros_like(a[0])
+    for j in range(bits - 1, -1, -1):
+        for i in range(n):
+            key = (key << 1) | ((a[i] >> j) & 1)
+    order = np.argsort(key, kind="stable")
+    return np.concatenate([np.arange(n_text), n_text + order]).astype(np.int64)
+
+
+def permute_tokens_ref(x, perm, inverse=False):
+    """Rows of x [B, H, L, d] reordered: out[:, :, i] = x[:, :, perm[i]], or
+    out[:, :, perm[i]] = x[:, :, i] with inverse."""
+    perm = np.asarray(perm)
+    if not inverse:
+        return x[:, :, perm]
+    out = np.empty_like(x)
+    out[:, :, perm] = x
+    return out
+
+
 def build_block_index_ref(block_mask):
     """CSR of a dense block mask [Hm, nqb, nkb]: rows are (h, qb) flattened
     h-major; row_ptr has Hm*nqb+1 entries (exclusive prefix sum of the row

@@ -22,6 +22,7 @@ using namespace rtb;
 
 namespace rtb {
 rt_status api_cuda_fail(cudaError_t e, const char* where);
+rt_status api_status_word(unsigned int** out);
 }
 
 namespace {
@@ -61,6 +62,8 @@ rt_status status_word(unsigned int** out) {
 
 // Records a CUDA error for rt_last_cuda_error (used by the other translation units).
 rt_status rtb::api_cuda_fail(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+// The device status word of the current device (for the other translation units).
+rt_status rtb::api_status_word(unsigned int** out) { return status_word(out); }
 
 namespace {
 

@@ -80,9 +80,24 @@ for _dens, _tag in ((0.25, "25"), (0.125, "12.5"), (0.0625, "6.25"), (0.03125, "
 # static block masks
 # ---------------------------------------------------------------------------
 
-def block_centroids(w: Workload):
+def token_coords(w: Workload, perm=None) -> np.ndarray:
+    """(f, y, x) grid coordinates of the token at each position [L, 3]; NaN for
+    text tokens.  perm (optional, [L]): position i holds raster token perm[i]
+    (raster = text tokens, then the grid with x fastest)."""
+    raster = np.arange(w.L) if perm is None else np.asarray(perm, dtype=np.int64)
+    out = np.full((w.L, 3), np.nan)
+    if w.grid is not None:
+        F, Y, X = w.grid
+        vis = raster >= w.n_text
+        r = raster[vis] - w.n_text
+        out[vis] = np.stack([r // (Y * X), (r // X) % Y, r % X], axis=1)
+    return out
+
+
+def block_centroids(w: Workload, perm=None):
     """Mean (f, y, x) of each block's visual tokens; NaN rows for text-only blocks.
-    Also returns the boolean 'holds a text token' per block."""
+    Also returns the boolean 'holds a text token' per block.  perm as in
+    token_coords (text tokens stay first, so the text blocks do not move)."""
     nb = w.nqb
     tok = np.arange(w.L)
     blk = tok // w.block
@@ -91,9 +106,8 @@ def block_centroids(w: Workload):
         has_text[np.unique(blk[: w.n_text])] = True
     cent = np.full((nb, 3), np.nan)
     if w.grid is not None:
-        F, Y, X = w.grid
-        vis = tok[w.n_text:] - w.n_text
-        f, y, x = vis // (Y * X), (vis // X) % Y, vis % X
+        coords_all = token_coords(w, perm)
+        f, y, x = (coords_all[w.n_text:, k] for k in range(3))
         coords = np.stack([f, y, x], axis=1).astype(np.float64)
         vb = blk[w.n_text:]
         sums = np.zeros((nb, 3))
@@ -104,14 +118,15 @@ def block_centroids(w: Workload):
     return cent, has_text
 
 
-def block_mask(w: Workload) -> np.ndarray:
-    """uint8 [1, nqb, nkb] static block mask shared by every batch and head."""
+def block_mask(w: Workload, perm=None) -> np.ndarray:
+    """uint8 [1, nqb, nkb] static block mask shared by every batch and head,
+    built on the token order perm (see token_coords; default raster)."""
     nb = w.nqb
     m = np.zeros((nb, nb), dtype=np.uint8)
     if w.diagonal:
         np.fill_diagonal(m, 1)
         return m[None]
-    cent, has_text = block_centroids(w)
+    cent, has_text = block_centroids(w, perm)
     text_blocks = np.nonzero(has_text)[0]
     visual = ~np.isnan(cent[:, 0])
     for qb in range(nb):

@@ -46,7 +46,7 @@ EXPORTED = (
     "rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
     "rt_check_device_error", "rt_status_string", "rt_last_cuda_error", "rt_set_wait_limit_ns",
     "rt_debug_wait_timeout", "rt_build_arch", "rt_schedule_step", "rt_schedule_capture",
-    "rt_cycle_graph_launch", "rt_cycle_graph_destroy",
+    "rt_cycle_graph_launch", "rt_cycle_graph_destroy", "rt_hilbert_token_order", "rt_permute_tokens",
 )
 
 
@@ -109,6 +109,8 @@ def load_library() -> ctypes.CDLL:
     lib.rt_schedule_capture.argtypes = [ctypes.POINTER(RtAttnDesc), ctypes.POINTER(RtSchedule), vpp, vpp, vpp,
                                         ctypes.POINTER(RtBlockIndex), vpp, vp, vp, vp, ctypes.POINTER(vp)]
     lib.rt_cycle_graph_launch.argtypes = [vp, vp]
+    lib.rt_hilbert_token_order.argtypes = [i32, i32, i32, i32, vp]
+    lib.rt_permute_tokens.argtypes = [ctypes.POINTER(RtAttnDesc), vp, vp, vp, i32, vp]
     lib.rt_cycle_graph_destroy.argtypes = [vp]
     lib.rt_check_device_error.argtypes = [vp]
     lib.rt_status_string.argtypes = [ctypes.c_int]
@@ -120,6 +122,7 @@ def load_library() -> ctypes.CDLL:
     lib.rt_build_arch.argtypes = []
     for name in ("rt_build_block_index", "rt_calibrate", "rt_sparse_step", "rt_calibrate_ex", "rt_sparse_step_ex",
                  "rt_schedule_step", "rt_schedule_capture", "rt_cycle_graph_launch", "rt_cycle_graph_destroy",
+                 "rt_hilbert_token_order", "rt_permute_tokens",
                  "rt_check_device_error",
                  "rt_set_wait_limit_ns", "rt_debug_wait_timeout", "rt_build_arch"):
         getattr(lib, name).restype = ctypes.c_int
@@ -349,3 +352,31 @@ class CycleGraph:
             self.close()
         except Exception:
             pass
+
+
+def rt_hilbert_token_order(n_text: int, F: int, Y: int, X: int) -> torch.Tensor:
+    """Host int32 [n_text + F*Y*X]: perm[i] = raster index of the token at
+    position i of the Hilbert order (text tokens first)."""
+    lib = load_library()
+    perm = torch.empty(n_text + F * Y * X, dtype=torch.int32)
+    _check(lib.rt_hilbert_token_order(int(n_text), int(F), int(Y), int(X), perm.data_ptr()),
+           "rt_hilbert_token_order")
+    return perm
+
+
+def rt_permute_tokens(src, perm, *, inverse: bool = False, dst=None, stream=None):
+    """dst[:, :, i] = src[:, :, perm[i]] (inverse=False) or
+    dst[:, :, perm[i]] = src[:, :, i] (inverse=True); src bf16 [B, H, L, d]."""
+    lib = load_library()
+    _require_cuda(src, perm, dst)
+    if src.dtype != torch.bfloat16 or src.dim() != 4:
+        raise ValueError("src must be a bf16 [B, H, L, d] tensor")
+    if perm.dtype != torch.int32 or perm.dim() != 1 or perm.numel() != src.shape[2] or not perm.is_contiguous():
+        raise ValueError("perm must be a contiguous int32 [L] tensor")
+    dst = torch.empty_like(src) if dst is None else dst
+    _same_layout(src, dst)
+    desc = _desc(src, 128, 0.0, torch.bfloat16)
+    _check(lib.rt_permute_tokens(ctypes.byref(desc), src.data_ptr(), dst.data_ptr(), perm.data_ptr(),
+                                 1 if inverse else 0, _stream_ptr(stream)),
+           "rt_permute_tokens")
+    return dst

@@ -8,6 +8,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from sparse_attention_diffusion_rt_b200 import build as rtbuild
@@ -139,3 +140,32 @@ def test_binding_refuses_without_cuda(lib):
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(RuntimeError):
         rt.rt_calibrate(q, q, q, None, block=128)
+
+
+@pytest.mark.parametrize("n_text,F,Y,X", [(0, 13, 30, 45), (226, 13, 30, 45), (0, 32, 45, 80), (256, 1, 64, 64),
+                                          (0, 1, 64, 64), (3, 5, 1, 7), (0, 1, 1, 1)])
+def test_hilbert_token_order_matches_oracle(lib, n_text, F, Y, X):
+    """The library's (host, C++) token order equals the oracle's on the
+    workload grids, bit for bit."""
+    from oracle import reference as ref
+    got = rt.rt_hilbert_token_order(n_text, F, Y, X).numpy()
+    np.testing.assert_array_equal(got, ref.hilbert_order_ref(n_text, F, Y, X))
+
+
+def test_token_order_validation_without_gpu(lib):
+    vp = ctypes.c_void_p
+    buf = (ctypes.c_int32 * 8)()
+    assert lib.rt_hilbert_token_order(0, 0, 2, 2, buf) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_hilbert_token_order(-1, 1, 2, 2, buf) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_hilbert_token_order(0, 1, 2, 2, None) == rt.RT_ERR_INVALID_ARGUMENT
+    desc = rt.RtAttnDesc(1, 1, 128, 64, 128, 8192, 8192, 64, 0.0, 0)
+    assert lib.rt_permute_tokens(ctypes.byref(desc), vp(4096), vp(8192), None, 0, None) == rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_permute_tokens(ctypes.byref(desc), vp(4096), vp(8192), vp(4096), 2, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                            # inverse must be 0 or 1
+    assert lib.rt_permute_tokens(ctypes.byref(desc), vp(4096), vp(4096), vp(64), 0, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                            # in place
+    assert lib.rt_permute_tokens(ctypes.byref(desc), vp(4096 + 8), vp(8192), vp(64), 0, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                            # misaligned
+    bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)
+    assert lib.rt_permute_tokens(ctypes.byref(bad), vp(4096), vp(8192), vp(64), 0, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                            # d % 8 != 0

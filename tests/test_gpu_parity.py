@@ -489,3 +489,57 @@ def test_host_validation_rejects_before_launch():
         rt.rt_calibrate(q, k, v, bad_idx, block=128)
     assert e.value.status == rt.RT_ERR_INVALID_ARGUMENT
     _ok()
+
+
+# ---------------------------------------------------------------------------
+# token reordering
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,L,d,strided", [(1, 2, 300, 72, False), (2, 3, 1000, 128, False), (2, 4, 256, 64, True)])
+def test_permute_tokens_bit_exact(B, H, L, d, strided):
+    g = torch.Generator(device=DEV).manual_seed(L + d)
+    if strided:                                      # [B, L, H, d] storage viewed as [B, H, L, d]
+        x = torch.randn((B, L, H, d), generator=g, device=DEV).to(torch.bfloat16).transpose(1, 2)
+    else:
+        x = torch.randn((B, H, L, d), generator=g, device=DEV).to(torch.bfloat16)
+    perm = torch.randperm(L, generator=g, device=DEV).to(torch.int32)
+    y = rt.rt_permute_tokens(x, perm)
+    z = rt.rt_permute_tokens(y, perm, inverse=True)
+    torch.cuda.synchronize()
+    _ok()
+    assert torch.equal(y, x[:, :, perm.long()])
+    assert torch.equal(z, x)
+
+
+def test_permute_tokens_bad_entry_recorded():
+    L = 200
+    x = torch.randn((1, 2, L, 64), device=DEV).to(torch.bfloat16)
+    perm = torch.arange(L, device=DEV, dtype=torch.int32)
+    perm[7] = L                                      # out of range: recorded, row skipped
+    y = torch.zeros_like(x)
+    rt.rt_permute_tokens(x, perm, dst=y)
+    assert rt.rt_check_device_error() == rt.RT_ERR_BAD_INDEX
+    keep = torch.ones(L, dtype=torch.bool, device=DEV)
+    keep[7] = False
+    assert torch.equal(y[:, :, keep], x[:, :, keep])
+    assert torch.count_nonzero(y[:, :, 7]) == 0
+
+
+def test_reordered_tokens_calibrate_and_sparse_step():
+    """Hilbert-ordered tokens with the block mask built on them: the GPU cycle
+    matches the oracle on the reordered problem, and with a dense mask the
+    reordered full attention scattered back equals raster full attention."""
+    w = inputs.Workload("grid", 1, 2, 4 * 8 * 16 + 64, 64, 128, kept=2, n_sparse_steps=1, seed=7,
+                        n_text=64, grid=(4, 8, 16))
+    perm_h = rt.rt_hilbert_token_order(w.n_text, *w.grid)
+    perm = perm_h.to(DEV)
+    (q, k, v), (q2, k2, v2) = inputs.qkv_steps(w, 2, device=DEV)
+    qp, kp, vp, q2p, k2p, v2p = (rt.rt_permute_tokens(t, perm) for t in (q, k, v, q2, k2, v2))
+    mask = inputs.block_mask(w, perm_h.numpy())
+    _run_cycle_full(qp, kp, vp, q2p, k2p, v2p, mask, w.block)
+    dense = np.ones((1, w.nqb, w.nkb), dtype=np.uint8)
+    o_p, _, _ = rt.rt_calibrate(qp, kp, vp, _index(dense), block=w.block)
+    o_back = rt.rt_permute_tokens(o_p, perm, inverse=True)
+    torch.cuda.synchronize()
+    _ok()
+    check_out(f64(o_back), ref.full_attention_ref(f64(q), f64(k), f64(v)), "reordered full attention, back")

@@ -350,3 +350,59 @@ def test_oracle_exports():
     for name in ("full_attention_ref", "calibrate_ref", "sparse_step_ref", "ramp_ref",
                  "build_block_index_ref", "ditfastattn_residual_ref"):
         assert callable(getattr(oracle, name))
+
+
+# ---------------------------------------------------------------------------
+# token reordering (Hilbert order of the latent grid)
+# ---------------------------------------------------------------------------
+
+def _grid_points(perm, n_text, F, Y, X):
+    r = np.asarray(perm[n_text:]) - n_text
+    return np.stack([r // (Y * X), (r // X) % Y, r % X], axis=1)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2), (1, 4, 4), (1, 8, 8), (1, 16, 16), (2, 2, 2), (4, 4, 4), (8, 8, 8)])
+def test_hilbert_order_is_a_unit_step_curve_on_full_cubes(shape):
+    """On a full 2^b cube the order is a Hamiltonian path of unit steps that
+    starts at the origin: the defining property of a Hilbert curve."""
+    perm = ref.hilbert_order_ref(0, *shape)
+    assert sorted(perm.tolist()) == list(range(int(np.prod(shape))))
+    pts = _grid_points(perm, 0, *shape)
+    assert (pts[0] == 0).all()
+    steps = np.abs(np.diff(pts, axis=0)).sum(axis=1)
+    assert (steps == 1).all()
+
+
+@pytest.mark.parametrize("shape,sub", [((8, 8, 8), 4), ((1, 16, 16), 4), ((16, 16, 16), 8)])
+def test_hilbert_order_visits_aligned_subcubes_contiguously(shape, sub):
+    """Consecutive runs of sub^n points are aligned sub-cubes: a block of the
+    reordered tokens is a compact brick, which is what the reordering is for."""
+    perm = ref.hilbert_order_ref(0, *shape)
+    pts = _grid_points(perm, 0, *shape)
+    n = sum(1 for e in shape if e > 1)
+    run = sub ** n
+    for s0 in range(0, len(pts), run):
+        chunk = pts[s0:s0 + run]
+        ext = chunk.max(axis=0) - chunk.min(axis=0) + 1
+        assert all(e == (sub if full > 1 else 1) for e, full in zip(ext, shape))
+        assert (chunk.min(axis=0) % sub == 0).all()
+
+
+def test_hilbert_order_keeps_text_first_and_restricts_the_cube():
+    perm = ref.hilbert_order_ref(5, 3, 6, 5)
+    assert perm[:5].tolist() == list(range(5))
+    assert sorted(perm.tolist()) == list(range(5 + 90))
+    # the order of a grid is the enclosing cube's order with the outside points dropped
+    cube = ref.hilbert_order_ref(0, 8, 8, 8)
+    cube_pts = _grid_points(cube, 0, 8, 8, 8)
+    inside = cube_pts[(cube_pts[:, 0] < 3) & (cube_pts[:, 1] < 6) & (cube_pts[:, 2] < 5)]
+    np.testing.assert_array_equal(_grid_points(perm, 5, 3, 6, 5), inside)
+
+
+def test_permute_tokens_ref_gathers_and_scatters():
+    x = np.arange(2 * 3 * 5 * 2).reshape(2, 3, 5, 2).astype(np.float64)
+    perm = np.array([3, 0, 4, 1, 2])
+    y = ref.permute_tokens_ref(x, perm)
+    for i in range(5):
+        np.testing.assert_array_equal(y[:, :, i], x[:, :, perm[i]])
+    np.testing.assert_array_equal(ref.permute_tokens_ref(y, perm, inverse=True), x)
