@@ -172,9 +172,10 @@ class Step:
     def __init__(self, w, mask_dev, qkv_steps, rt):
         self.w, self.mask, self.qkv, self.rt = w, mask_dev, qkv_steps, rt
         q = qkv_steps[0][0]
-        self.o = [torch.empty_like(q) for _ in qkv_steps]
+        like_q = lambda: torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device)
+        self.o = [like_q() for _ in qkv_steps]          # same strides as the inputs (head-shard views too)
         self.rho = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=q.device)
-        self.r = torch.empty_like(q)
+        self.r = like_q()
         n = len(qkv_steps)
         self.ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         self.times = {"calibrate": [], "sparse": []}
@@ -424,12 +425,23 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     n_steps = 1 + w.n_sparse_steps
     qkv = inputs.qkv_steps(w, n_steps, device=dev)
+    w_job = w
+    sharded = args.shard == "heads" and world > 1
+    if sharded:
+        # one problem split by heads: this rank's heads as strided views, no collective
+        from sparse_attention_diffusion_rt_b200 import shard
+        h0, h1 = shard.head_range(w.H, world, rank)
+        qkv = [tuple(shard.shard_heads(x, h0, h1) for x in s) for s in qkv]
+        w = dataclasses.replace(w, H=h1 - h0)
     mask_np = inputs.block_mask(w)
     mask = torch.from_numpy(mask_np).to(dev)
     nnz = int(mask_np.sum())
     cal_flops = executed_flops(w, w.nqb * w.nkb)
     sp_flops = executed_flops(w, nnz)
     step_flops = cal_flops + w.n_sparse_steps * sp_flops
+    # whole-job work per step: N replicas, or the one problem the shards split
+    job_step_flops = (executed_flops(w_job, w.nqb * w.nkb) + w.n_sparse_steps * executed_flops(w_job, nnz)
+                      if sharded else world * step_flops)
     step = Step(w, mask, qkv, rt)
 
     def barrier():
@@ -465,7 +477,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error in timed region: {rt.rt_status_string(st)}")
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = job_tflops(world, step_flops, ms_per_step)
+    value = job_tflops(1, job_step_flops, ms_per_step)
 
     # ---- per-kernel timing: separate pass, each kernel bracketed by events
     step.times = {"calibrate": [], "sparse": []}
@@ -565,7 +577,7 @@ def run_ours(args, rank, world, local_rank):
         e_ms = max_over_ranks(e_ms, world, dev)
         # the outputs read back equal the device-resident path's on the same inputs
         match = all(torch.equal(ho, o.cpu()) for ho, o in zip(host_out, step.o))
-        e2e = {"value": job_tflops(world, step_flops, e_ms), "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(1, job_step_flops, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "copies": "H2D and D2H on their own streams, 2 device buffer sets, overlapping the kernels",
                "outputs_match_device_path": bool(match)}
@@ -592,14 +604,14 @@ def run_ours(args, rank, world, local_rank):
         sdpa = {"error": str(exc)[:200]}
 
     schedule = None
-    if not args.no_schedule:
+    if not args.no_schedule and not sharded:
         try:
             schedule = measure_schedule(w, mask, rt)
         except torch.cuda.OutOfMemoryError as exc:
             schedule = {"error": str(exc)[:200]}
 
     token_order = None
-    if not args.no_schedule:
+    if not args.no_schedule and not sharded:
         token_order = measure_token_order(w, rt)
 
     cpu = None
@@ -611,12 +623,14 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block,
+            "config": {"workload": w_job.name, "B": w_job.B, "H": w_job.H, "L": w.L, "d": w.d, "block": w.block,
                        "kept_blocks_per_row": w.kept, "sparsity": 1 - nnz / (w.nqb * w.nkb),
                        "sparse_steps": w.n_sparse_steps, "lambda": w.lam,
-                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+                       "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"heads x{world} (one problem)" if sharded else f"replicas x{world}"},
             "step": "block index + 1 calibration + %d sparse steps" % w.n_sparse_steps,
             "sparse_step": {"latency_us": sp_ms * 1e3, "tflops": sp_tf, "frac_of_peak": sp_tf / peak,
                             "executed_gflop": sp_flops / 1e9},
@@ -647,6 +661,8 @@ def main():
     ap.add_argument("--no-schedule", action="store_true",
                     help="skip the denoising-schedule and token-order measurements")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas (weak scaling, default) or one problem split by heads")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (a smaller case for profiling)")
     args = ap.parse_args()

@@ -212,7 +212,7 @@ def rt_calibrate(q, k, v, index: BlockIndex, *, block: int, o=None, rho=None, r=
         if t.dtype != torch.bfloat16:
             raise ValueError("q, k, v must be bfloat16")
     B, H, L, d = q.shape
-    o = torch.empty_like(q) if o is None else o
+    o = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if o is None else o
     r = torch.empty_strided(q.shape, q.stride(), dtype=r_dtype, device=q.device) if r is None else r
     rho = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if rho is None else rho
     if o.dtype != torch.bfloat16 or r.dtype != r_dtype or rho.dtype != torch.float32 or not rho.is_contiguous():
@@ -245,7 +245,7 @@ def rt_sparse_step(q, k, v, index: BlockIndex, rho, r, *, block: int, lam: float
         raise ValueError("r must be bf16 or fp32")
     if rho is not None and (rho.dtype != torch.float32 or not rho.is_contiguous()):
         raise ValueError("rho must be fp32 contiguous [B, H, L]")
-    o = torch.empty_like(q) if o is None else o
+    o = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if o is None else o
     if o.dtype != torch.bfloat16:
         raise ValueError("o must be bfloat16")
     _same_layout(q, k, v, o, *(() if r is None else (r,)))

@@ -543,3 +543,32 @@ def test_reordered_tokens_calibrate_and_sparse_step():
     torch.cuda.synchronize()
     _ok()
     check_out(f64(o_back), ref.full_attention_ref(f64(q), f64(k), f64(v)), "reordered full attention, back")
+
+
+# ---------------------------------------------------------------------------
+# head sharding
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("per_head_mask,d", [(False, 128), (True, 64), (True, 88)])
+def test_head_shards_reproduce_the_whole_problem(per_head_mask, d):
+    """Each rank of a head-sharded run calls the library on strided views of
+    its heads (and the slice of a per-head mask); the pieces equal the
+    unsharded outputs exactly, since heads are independent."""
+    from sparse_attention_diffusion_rt_b200 import shard
+    B, H, L, blk, world = 2, 5, 3 * 128 - 20, 128, 2
+    q, k, v = inputs.random_qkv(B, H, L, d, seed=120 + d, device=DEV)
+    q2, k2, v2 = inputs.random_qkv(B, H, L, d, seed=121 + d, device=DEV)
+    mask = inputs.random_block_mask(H if per_head_mask else 1, 3, 3, 0.5, seed=122, ensure_nonempty=True)
+    idx = _index(mask)
+    o, rho, r = rt.rt_calibrate(q, k, v, idx, block=blk)
+    o2 = rt.rt_sparse_step(q2, k2, v2, idx, rho, r, block=blk, step_distance=2)
+    for rank in range(world):
+        h0, h1 = shard.head_range(H, world, rank)
+        sl = lambda t: shard.shard_heads(t, h0, h1)
+        idx_s = _index(shard.shard_mask(mask, h0, h1))
+        o_s, rho_s, r_s = rt.rt_calibrate(sl(q), sl(k), sl(v), idx_s, block=blk)
+        o2_s = rt.rt_sparse_step(sl(q2), sl(k2), sl(v2), idx_s, rho_s, r_s, block=blk, step_distance=2)
+        torch.cuda.synchronize()
+        _ok()
+        assert torch.equal(o_s, sl(o)) and torch.equal(rho_s, sl(rho)) and torch.equal(r_s, sl(r))
+        assert torch.equal(o2_s, sl(o2))

@@ -10,6 +10,8 @@ the other ranks exit without work.
 import os
 import socket
 
+import numpy as np
+
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -80,3 +82,63 @@ def test_reference_arm_runs_on_rank_zero_only():
         warmup = 3
     # a non-zero rank returns at once, without touching the oracle or printing a line
     assert bench.run_reference(Args(), rank=1, world=2) is None
+
+
+def test_head_ranges_partition_the_heads():
+    from sparse_attention_diffusion_rt_b200 import shard
+    for H in (1, 7, 16, 24, 30):
+        for world in (1, 2, 3, 4, 8):
+            if world > H:
+                continue
+            ranges = [shard.head_range(H, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))      # contiguous, no overlap
+            sizes = [h1 - h0 for h0, h1 in ranges]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    with pytest.raises(ValueError):
+        shard.head_range(4, 2, 2)
+
+
+def test_shard_mask_slices_per_head_masks_only():
+    from sparse_attention_diffusion_rt_b200 import shard
+    shared = np.ones((1, 3, 3), np.uint8)
+    assert shard.shard_mask(shared, 2, 5) is shared
+    per_head = np.arange(6 * 2 * 2).reshape(6, 2, 2).astype(np.uint8)
+    np.testing.assert_array_equal(shard.shard_mask(per_head, 2, 5), per_head[2:5])
+
+
+def _shard_rank_main(rank, world, port, H, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    from sparse_attention_diffusion_rt_b200 import shard
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    try:
+        h0, h1 = shard.head_range(H, world, rank)
+        counts = torch.zeros(H, dtype=torch.int64)
+        counts[h0:h1] = 1
+        torch.distributed.all_reduce(counts)                   # every head owned by exactly one rank
+        out[rank] = counts.tolist()
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_head_sharding_gloo_every_head_once():
+    world, H = 2, 7
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_shard_rank_main, args=(r, world, port, H, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+                p.join()
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    assert res[0] == res[1] == [1] * H
