@@ -13,17 +13,19 @@
 //              and the residual tile; lane 1 loads the V tiles.  K and V have
 //              their own NST-stage rings, released after QK^T and after PV.
 //   warp 5     lane 0 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
-//              logit buffers, O += P V with P read from TMEM.  The QK^T of
-//              block j+2 is issued as soon as the softmax has read block j's
-//              logits, so the tensor pipe always has the next logits ready.
+//              logit buffers, O += P V with P read from TMEM.  The softmax
+//              writes P over its own logits, so the MMA warp issues PV(j) and
+//              then QK^T(j+2) into the same buffer: MMAs of one thread run in
+//              issue order, so the logits are never overwritten early and the
+//              tensor pipe always has the next logits queued.
 // Tile metadata flows through a 2-slot ring (ti_*).  Every per-block barrier
 // phase is indexed by a block counter that runs across tiles, so the MMA warp
 // starts the next tile's QK^T while the softmax warps finish the previous
 // tile's epilogue; the output leaves through a shared-memory staging tile and
 // a TMA store that is only waited for when its staging slot comes round again.
 //
-// TMEM columns: S0/S1 [0,256) fp32 logits, P0/P1 [256,384) bf16
-// probabilities, O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
+// TMEM columns: S0/S1 [0,256) fp32 logits, each overwritten in place by its
+// bf16 probabilities P (64 columns of the 128), O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
 // and every role drains what it has in flight before TMEM is freed.
 #pragma once
 #include <cuda.h>
@@ -52,7 +54,7 @@ struct SpCfg {
   static constexpr int OFF_OST = OFF_R + TILE_BYTES;
   static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static constexpr uint32_t T_S = 0, T_P = 256, T_O = 384;   // S_b at 128b, P_b at 256 + 64b
+  static constexpr uint32_t T_S = 0, T_O = 384;   // S_b (and P_b over it) at 128b, O at 384
 };
 
 struct SpTile {
@@ -63,7 +65,7 @@ struct SpTile {
 struct SpCtrl {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full;
   uint64_t r_full, r_empty;
   uint64_t ti_full[2], ti_empty[2];
@@ -217,11 +219,11 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
   uint32_t g = 0, qi = 0;
   bool ok = true;
 
-  // S_(gi&1) = Q K_gi^T once the softmax has read the logits two blocks back
+  // S_(gi&1) = Q K_gi^T.  It overwrites P(gi-2) (P is written over its own
+  // logits), whose PV was issued before: MMAs of one thread run in issue order.
   auto issue_qk = [&](uint32_t gi, uint32_t q_addr) -> bool {
     const int st = gi % C::NST;
     if (!sp_wait(&ctl.k_full[st], (gi / C::NST) & 1, ctl, p)) return false;
-    if (gi >= 2 && !sp_wait(&ctl.s_free[gi & 1], ((gi >> 1) - 1) & 1, ctl, p)) return false;
     tc_fence_after();
     const uint32_t k_tile = stage0 + st * C::STAGE_BYTES;
     const uint32_t dst = tmem + C::T_S + 128u * (gi & 1);
@@ -238,7 +240,7 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
     if (!sp_wait(&ctl.v_full[st], (gi / C::NST) & 1, ctl, p)) return false;
     tc_fence_after();
     const uint32_t v_tile = stage0 + st * C::STAGE_BYTES + C::TILE_BYTES;
-    const uint32_t tp = tmem + C::T_P + 64u * (gi & 1);
+    const uint32_t tp = tmem + C::T_S + 128u * (gi & 1);
     const uint32_t dst = tmem + C::T_O;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
@@ -263,13 +265,15 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
       const uint32_t q_addr = q0 + qs * C::TILE_BYTES;
       const uint32_t g0 = g;
       for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_qk(g0 + i, q_addr);
+      if (ok && n <= 2) mma_commit(&ctl.q_empty[qs]);          // the tile's last QK^T has been issued
       for (int j = 0; ok && j < n; ++j) {
-        if (j + 2 < n) ok = issue_qk(g0 + j + 2, q_addr);
-        if (ok && j + 2 == n) mma_commit(&ctl.q_empty[qs]);   // the tile's last QK^T has been issued
-        if (ok) ok = issue_pv(g0 + j, j == 0);
+        ok = issue_pv(g0 + j, j == 0);
+        if (ok && j + 2 < n) {
+          ok = issue_qk(g0 + j + 2, q_addr);
+          if (ok && j + 3 == n) mma_commit(&ctl.q_empty[qs]);
+        }
       }
       if (!ok) break;
-      if (n == 1) mma_commit(&ctl.q_empty[qs]);
       mma_commit(&ctl.o_full);
       g = g0 + n;
       ++qi;
@@ -317,14 +321,17 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       uint32_t s[128];
       load_scores<128>(tS + 128u * bf, s);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&ctl.s_free[bf]);
       mask_tail<128>(s, (j == ti.tail_j) ? ti.tail_valid : 128);
-      const float mx = row_max<128>(s) * sl2;
-      if (j == 0) {
-        m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
-        const float m_new = fmaxf(m, mx);
+      if (j == 0) m = row_max<128>(s) * sl2;
+      // P(g) over the first 64 columns of its own logits (they are in registers),
+      // with the running max; xmax, the block's largest s * sl2 - m, tells
+      // whether that max was too small
+      float xmax;
+      float sum = exp_pack_store_mx<128>(s, sl2, m, tS + 128u * bf, xmax);
+      if (__any_sync(0xffffffffu, xmax > kRescaleLog2)) {
+        // rare: the block raised the max by more than 2^8: rescale O, then redo P(g)
+        tmem_wait_st();                       // the first P(g) stores land before they are redone
+        const float m_new = m + fmaxf(xmax, 0.f);
         const float alpha = ex2_approx(m - m_new);
         l *= alpha;
         // O holds blocks up to g-1: wait for PV(g-1)
@@ -333,14 +340,9 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
         tc_fence_after();
         rescale_row<DPAD>(tO, alpha);
         m = m_new;
+        sum = exp_pack_store<128>(s, sl2, m, tS + 128u * bf);
       }
-      // P buffer bf was last read by PV(g-2)
-      if (g >= 2) {
-        ok = __all_sync(0xffffffffu, sp_wait(&ctl.pv_done[bf], ((g >> 1) - 1) & 1, ctl, p));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      l += exp_pack_store<128>(s, sl2, m, tmem + lane_base + C::T_P + 64u * bf);
+      l += sum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ctl.p_full[bf]);
@@ -452,7 +454,6 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
       mbar_init(&ctl.q_full[i], 1);
       mbar_init(&ctl.q_empty[i], 1);
       mbar_init(&ctl.s_full[i], 1);
-      mbar_init(&ctl.s_free[i], kSoftmaxThreads);
       mbar_init(&ctl.p_full[i], kSoftmaxThreads);
       mbar_init(&ctl.pv_done[i], 1);
       mbar_init(&ctl.ti_full[i], 1);
