@@ -140,6 +140,14 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// TMEM lanes 0..127, 8 columns from `taddr` <- a 128-row x 32-byte shared-memory
+// matrix given by an operand descriptor (row r to lane r, its bytes in order, so
+// bf16 pairs land in 32-bit columns as a TMEM A operand wants them).  Asynchronous;
+// a later tcgen05.mma of the same thread sees the copy (the pair runs in issue
+// order) and tcgen05.commit tracks its completion.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"

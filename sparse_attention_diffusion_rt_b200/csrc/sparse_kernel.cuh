@@ -12,8 +12,10 @@
 //              (double-buffered for d <= 96), the K tiles of the kept blocks
 //              and the residual tile; lane 1 loads the V tiles.  K and V have
 //              their own NST-stage rings, released after QK^T and after PV.
-//   warp 5     lane 0 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
-//              logit buffers, O += P V with P read from TMEM.  The softmax
+//   warp 5     lane 0 issues the tcgen05 MMAs: it copies each tile's Q into
+//              TMEM (tcgen05.cp), then S = Q K^T into one of two TMEM logit
+//              buffers with Q read from TMEM, O += P V with P read from TMEM,
+//              so only K and V are read from shared memory.  The softmax
 //              writes P over its own logits, so the MMA warp issues PV(j) and
 //              then QK^T(j+2) into the same buffer: MMAs of one thread run in
 //              issue order, so the logits are never overwritten early and the
@@ -25,7 +27,8 @@
 // a TMA store that is only waited for when its staging slot comes round again.
 //
 // TMEM columns: S0/S1 [0,256) fp32 logits, each overwritten in place by its
-// bf16 probabilities P (64 columns of the 128), O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
+// bf16 probabilities P (64 columns of the 128), Q [256, 256+DPAD/2) as bf16
+// pairs, O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
 // and every role drains what it has in flight before TMEM is freed.
 #pragma once
 #include <cuda.h>
@@ -54,7 +57,8 @@ struct SpCfg {
   static constexpr int OFF_OST = OFF_R + TILE_BYTES;
   static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static constexpr uint32_t T_S = 0, T_O = 384;   // S_b (and P_b over it) at 128b, O at 384
+  static constexpr uint32_t T_S = 0, T_Q = 256, T_O = 384;   // S_b (and P_b over it) at 128b, Q, O
+  static_assert(T_Q + DPAD / 2 <= T_O, "Q (bf16 pairs) fits below O");
 };
 
 struct SpTile {
@@ -221,7 +225,8 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
 
   // S_(gi&1) = Q K_gi^T.  It overwrites P(gi-2) (P is written over its own
   // logits), whose PV was issued before: MMAs of one thread run in issue order.
-  auto issue_qk = [&](uint32_t gi, uint32_t q_addr) -> bool {
+  // Q is read from its TMEM copy (A operand), K from shared memory.
+  auto issue_qk = [&](uint32_t gi) -> bool {
     const int st = gi % C::NST;
     if (!sp_wait(&ctl.k_full[st], (gi / C::NST) & 1, ctl, p)) return false;
     tc_fence_after();
@@ -229,7 +234,7 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
     const uint32_t dst = tmem + C::T_S + 128u * (gi & 1);
 #pragma unroll
     for (int kk = 0; kk < DPAD / 16; ++kk)
-      mma_ss(dst, kmajor_desc<DPAD>(q_addr, 128, kk), kmajor_desc<DPAD>(k_tile, 128, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+      mma_ts(dst, tmem + C::T_Q + kk * 8, kmajor_desc<DPAD>(k_tile, 128, kk), IDESC_QK, kk > 0 ? 1u : 0u);
     mma_commit(&ctl.s_full[gi & 1]);
     mma_commit(&ctl.k_empty[st]);
     return true;
@@ -262,16 +267,20 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
     if (n > 0) {
       const int qs = C::QBUF == 2 ? (qi & 1) : 0;
       if (!sp_wait(&ctl.q_full[qs], (qi / C::QBUF) & 1, ctl, p)) { ok = false; break; }
+      // Q tile -> TMEM.  Every QK^T of the previous tile has completed (its last
+      // PV waited for the softmax, which had read the last logits), so the one
+      // TMEM copy of Q is free; the shared-memory buffer is released as soon as
+      // the copy is done.
+      tc_fence_after();
       const uint32_t q_addr = q0 + qs * C::TILE_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < DPAD / 16; ++kk) tmem_cp_128x256b(tmem + C::T_Q + kk * 8, kmajor_desc<DPAD>(q_addr, 128, kk));
+      mma_commit(&ctl.q_empty[qs]);
       const uint32_t g0 = g;
-      for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_qk(g0 + i, q_addr);
-      if (ok && n <= 2) mma_commit(&ctl.q_empty[qs]);          // the tile's last QK^T has been issued
+      for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_qk(g0 + i);
       for (int j = 0; ok && j < n; ++j) {
         ok = issue_pv(g0 + j, j == 0);
-        if (ok && j + 2 < n) {
-          ok = issue_qk(g0 + j + 2, q_addr);
-          if (ok && j + 3 == n) mma_commit(&ctl.q_empty[qs]);
-        }
+        if (ok && j + 2 < n) ok = issue_qk(g0 + j + 2);
       }
       if (!ok) break;
       mma_commit(&ctl.o_full);
