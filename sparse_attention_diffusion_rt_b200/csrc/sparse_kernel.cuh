@@ -358,54 +358,12 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
     }
     if (!ok) break;
     // ------------------------------------------------------------- epilogue
-    if (ti.n > 0) {
-      ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_full, oi & 1, ctl, p));
-      if (!ok) break;
-      tc_fence_after();
-      ++oi;
-    }
-    if (!p.r_f32 && p.use_r) {
+    // The waits that do not need O (the residual tile, the staging slot) are
+    // taken while the tile's last PV runs.
+    const bool r_smem = !p.r_f32 && p.use_r;
+    if (r_smem) {
       ok = __all_sync(0xffffffffu, sp_wait(&ctl.r_full, ri & 1, ctl, p));
       if (!ok) break;
-    }
-    const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
-    const float scale = ti.n > 0 ? rho_hat / l : 0.f;
-    uint32_t packed[DPAD / 2];
-#pragma unroll
-    for (int c = 0; c < DPAD; c += 16) {
-      uint32_t acc[16];
-      if (ti.n > 0) { tmem_ld_x16(tO + c, acc); tmem_wait_ld(); }
-      float rr[16];
-      if (!p.use_r) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) rr[i] = 0.f;
-      } else if (p.r_f32) {
-        if (grow < p.L) {
-          const float4* src = reinterpret_cast<const float4*>(
-              static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
-              static_cast<long long>(grow) * p.stride_l + c);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4 v4 = (c + 4 * u < p.d) ? __ldg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-            rr[4 * u] = v4.x; rr[4 * u + 1] = v4.y; rr[4 * u + 2] = v4.z; rr[4 * u + 3] = v4.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rr[i] = 0.f;
-        }
-      } else {
-        load_row16<DPAD>(sR, 128, t, c, false, rr);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float a0 = (ti.n > 0 ? __uint_as_float(acc[2 * i]) * scale : 0.f) + rr[2 * i];
-        const float a1 = (ti.n > 0 ? __uint_as_float(acc[2 * i + 1]) * scale : 0.f) + rr[2 * i + 1];
-        packed[c / 2 + i] = pack_bf16x2(a0, a1);
-      }
-    }
-    if (!p.r_f32 && p.use_r) {
-      mbar_arrive(&ctl.r_empty);
-      ++ri;
     }
     // staging slot: thread 0 makes sure the store that last used it has read it
     const int ss = C::OSTG == 2 ? (si & 1) : 0;
@@ -413,24 +371,62 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       if (C::OSTG == 2) tma_store_wait_read<1>(); else tma_store_wait_read<0>();
       mbar_arrive(&ctl.stg_ready);
     }
+    if (ti.n > 0) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_full, oi & 1, ctl, p));
+      if (!ok) break;
+      tc_fence_after();
+      ++oi;
+    }
+    const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
+    const float scale = ti.n > 0 ? rho_hat / l : 0.f;
     ok = __all_sync(0xffffffffu, sp_wait(&ctl.stg_ready, si & 1, ctl, p));
     if (!ok) break;
     uint8_t* ost = sOst + ss * C::TILE_BYTES;
+    // 16 columns at a time: O from TMEM, the residual, the bf16 result into the
+    // staging tile (reading more of O per wait measured slower: it spills)
 #pragma unroll
     for (int c = 0; c < DPAD; c += 16) {
+      uint32_t acc[16];
+      if (ti.n > 0) {
+        tmem_ld_x16(tO + c, acc);
+        tmem_wait_ld();
+      }
+      float rr[16];
+      if (r_smem) {
+        load_row16<DPAD>(sR, 128, t, c, false, rr);
+      } else if (p.use_r && grow < p.L) {
+        // fp32 residual straight from global memory
+        const float4* src = reinterpret_cast<const float4*>(
+            static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
+            static_cast<long long>(grow) * p.stride_l + c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 v4 = (c + 4 * u < p.d) ? __ldg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+          rr[4 * u] = v4.x; rr[4 * u + 1] = v4.y; rr[4 * u + 2] = v4.z; rr[4 * u + 3] = v4.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rr[i] = 0.f;
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a0 = (ti.n > 0 ? __uint_as_float(acc[2 * i]) * scale : 0.f) + rr[2 * i];
+        const float a1 = (ti.n > 0 ? __uint_as_float(acc[2 * i + 1]) * scale : 0.f) + rr[2 * i + 1];
+        pk[i] = pack_bf16x2(a0, a1);
+      }
       const bool c1 = c >= 64;
       const uint32_t rb = c1 ? C::C1B : 128;
       const uint32_t cbase = c1 ? 128 * 128 : 0;
       const int col = c1 ? c - 64 : c;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        uint4 w;
-        w.x = packed[c / 2 + 4 * u + 0];
-        w.y = packed[c / 2 + 4 * u + 1];
-        w.z = packed[c / 2 + 4 * u + 2];
-        w.w = packed[c / 2 + 4 * u + 3];
-        *reinterpret_cast<uint4*>(ost + cbase + swz_off(t * rb + (col * 2 + u * 16), rb)) = w;
-      }
+      for (int u = 0; u < 2; ++u)
+        *reinterpret_cast<uint4*>(ost + cbase + swz_off(t * rb + (col * 2 + u * 16), rb)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+    }
+    if (r_smem) {
+      mbar_arrive(&ctl.r_empty);
+      ++ri;
     }
     fence_proxy_async_smem();
     mbar_arrive(&ctl.stg_full);
