@@ -9,9 +9,10 @@
 // + i * gridDim.x, query block fastest (see sp_decode).  Roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
 //   warp 4     producer: lane 0 validates each tile's CSR row and loads Q
-//              (double-buffered for d <= 96), the K tiles of the kept blocks
-//              and the residual tile; lane 1 loads the V tiles.  K and V have
-//              their own NST-stage rings, released after QK^T and after PV.
+//              (one buffer, free again once Q is in TMEM), the K tiles of the
+//              kept blocks and the residual tile; lane 1 loads the V tiles.  K
+//              and V have their own NST-stage rings, released after QK^T and
+//              after PV.
 //   warp 5     lane 0 issues the tcgen05 MMAs: it copies each tile's Q into
 //              TMEM (tcgen05.cp), then S = Q K^T into one of two TMEM logit
 //              buffers with Q read from TMEM, O += P V with P read from TMEM,
@@ -46,16 +47,21 @@ struct SpCfg {
   static constexpr int C1 = DPAD - 64;
   static constexpr int C1B = C1 * 2;
   static constexpr uint32_t C1SWZ = C1 == 16 ? SWZ_32B : (C1 == 32 ? SWZ_64B : SWZ_128B);
-  static constexpr int QBUF = DPAD <= 96 ? 2 : 1;
-  static constexpr int NST = DPAD <= 80 ? 3 : 2;
-  static constexpr int OSTG = DPAD <= 96 ? 2 : 1;
+  // Q is copied into TMEM at the start of its tile, so one shared-memory buffer
+  // is enough; the rest goes to the K/V ring (4 stages at DPAD 80, 3 at 96, 2 at
+  // 128) and one output staging tile.
+  static constexpr int QBUF = 1;
+  static constexpr int OSTG = 1;
   static constexpr int TILE_BYTES = 128 * DPAD * 2;          // one bf16 [128][DPAD] tile
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;          // K + V
   static constexpr int OFF_Q = 1024;
   static constexpr int OFF_STAGE = OFF_Q + QBUF * TILE_BYTES;
+  static constexpr int NST_FIT = (232448 - 1024 - OFF_STAGE - (1 + OSTG) * TILE_BYTES) / STAGE_BYTES;
+  static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int OFF_R = OFF_STAGE + NST * STAGE_BYTES;
   static constexpr int OFF_OST = OFF_R + TILE_BYTES;
   static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
+  static_assert(NST >= 2, "at least two K/V stages");
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static constexpr uint32_t T_S = 0, T_Q = 256, T_O = 384;   // S_b (and P_b over it) at 128b, Q, O
   static_assert(T_Q + DPAD / 2 <= T_O, "Q (bf16 pairs) fits below O");
@@ -68,7 +74,7 @@ struct SpTile {
 
 struct SpCtrl {
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
+  uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full;
   uint64_t r_full, r_empty;
@@ -464,7 +470,7 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
       mbar_init(&ctl.ti_full[i], 1);
       mbar_init(&ctl.ti_empty[i], kSoftmaxThreads + 2);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&ctl.k_full[i], 1);
       mbar_init(&ctl.v_full[i], 1);
       mbar_init(&ctl.k_empty[i], 1);
