@@ -387,7 +387,7 @@ def _sample_rows(L, block, rng, n_mid=6):
     return np.array(sorted(set(rows)))
 
 
-@pytest.mark.parametrize("name", ["cogvideox", "longvideo-3.1", "longvideo-25"])
+@pytest.mark.parametrize("name", ["cogvideox", "longvideo-3.1", "longvideo-6.25", "longvideo-12.5", "longvideo-25"])
 def test_full_size_sampled_rows(name):
     w = inputs.WORKLOADS[name]
     steps = inputs.qkv_steps(w, 2, device=DEV)
