@@ -34,6 +34,11 @@
  *     128 inside the kernels), block in {64, 128}, strides multiples of 8
  *     elements, pointers 16-byte aligned, 1 <= L and ceil(L/block) <= 4096.
  *     Other shapes return RT_ERR_UNSUPPORTED.
+ *   - The strides must give every (b, h, l) row its own d elements (any
+ *     permuted dense layout, e.g. [B,H,L,d] or [B,L,H,d], or a slice of one);
+ *     a layout whose heads or batches alias returns RT_ERR_INVALID_ARGUMENT,
+ *     and so does a call whose outputs (O; rho and R where the call writes
+ *     them) overlap one of its inputs or each other.
  */
 #ifndef RT_B200_H
 #define RT_B200_H
@@ -221,10 +226,14 @@ RT_API rt_status rt_hilbert_token_order(int32_t n_text, int32_t F, int32_t Y, in
  * `desc`; B, H, L, d and the strides are used, the rest ignored):
  *   inverse = 0: dst[b, h, i, :] = src[b, h, perm[i], :]   (raster -> new order)
  *   inverse = 1: dst[b, h, perm[i], :] = src[b, h, i, :]   (back to raster order)
- * d_perm: device i32 [L], a permutation of 0..L-1.  An entry outside [0, L)
- * records RT_ERR_BAD_INDEX in the device status word and its row is skipped.
- * src and dst must not overlap.  d % 8 == 0, 16-byte aligned pointers and
- * strides that are multiples of 8 elements.  Asynchronous on `stream`. */
+ * d_perm: device i32 [L], a permutation of 0..L-1 (a bijection).  An entry
+ * outside [0, L) records RT_ERR_BAD_INDEX in the device status word and its
+ * row is skipped; a repeated entry is not detected (the gather copies that row
+ * twice; the scatter, inverse = 1, writes one dst row twice and leaves another
+ * unwritten).  src and dst must not overlap and the layout's rows must be
+ * disjoint (RT_ERR_INVALID_ARGUMENT otherwise).  d % 8 == 0, 16-byte aligned
+ * pointers and strides that are multiples of 8 elements.  Asynchronous on
+ * `stream`. */
 RT_API rt_status rt_permute_tokens(const rt_attn_desc* desc, const void* src, void* dst, const int32_t* d_perm,
                             int32_t inverse, void* stream);
 

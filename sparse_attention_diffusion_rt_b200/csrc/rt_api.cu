@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "attn_launch.h"
+#include "layout.h"
 #include "rt.h"
 
 namespace rtb {
@@ -140,9 +141,10 @@ rt_status make_residual_maps(CUtensorMap (&m)[4], const void* ptr, const rt_attn
 }
 
 // need_rho / need_r: whether the call reads (or writes) rho and R.
+// stats_out: the call writes rho and R (calibration) rather than reading them.
 rt_status validate(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                    const rt_block_index* idx, const void* o, const void* rho, const void* r,
-                   bool need_rho = true, bool need_r = true) {
+                   bool stats_out, bool need_rho = true, bool need_r = true) {
   if (!desc || !idx || !q || !k || !v || !o) return RT_ERR_INVALID_ARGUMENT;
   if ((need_rho && !rho) || (need_r && !r)) return RT_ERR_INVALID_ARGUMENT;
   const rt_attn_desc& d = *desc;
@@ -168,6 +170,22 @@ rt_status validate(const rt_attn_desc* desc, const void* q, const void* k, const
   // strides below 2^40 bytes (tensor-map limit)
   const long long lim = 1ll << 38;
   if (d.stride_b >= lim || d.stride_h >= lim || d.stride_l >= lim) return RT_ERR_UNSUPPORTED;
+  // distinct (b, h, l) rows must not share elements: different CTAs store them
+  if (!layout_rows_disjoint(d)) return RT_ERR_INVALID_ARGUMENT;
+  // what the call writes overlaps nothing else it reads or writes
+  const long long span2 = layout_span_bytes(d, 2);
+  const long long span_r = layout_span_bytes(d, d.r_dtype == RT_F32 ? 4 : 2);
+  const long long span_rho = static_cast<long long>(d.B) * d.H * d.L * 4;
+  const void* ins[3] = {q, k, v};
+  for (const void* in : ins) {
+    if (ranges_overlap(o, span2, in, span2)) return RT_ERR_INVALID_ARGUMENT;
+    if (stats_out && (ranges_overlap(r, span_r, in, span2) || ranges_overlap(rho, span_rho, in, span2)))
+      return RT_ERR_INVALID_ARGUMENT;
+  }
+  if (ranges_overlap(o, span2, need_r ? r : nullptr, span_r) ||
+      ranges_overlap(o, span2, need_rho ? rho : nullptr, span_rho) ||
+      (need_r && need_rho && ranges_overlap(r, span_r, rho, span_rho)))
+    return RT_ERR_INVALID_ARGUMENT;
   return RT_OK;
 }
 
@@ -271,7 +289,7 @@ rt_status rt_calibrate_ex(const rt_attn_desc* desc, const void* q, const void* k
                           const rt_block_index* idx, void* o, float* rho, void* r, rt_residual kind,
                           void* stream) {
   if (kind != RT_RES_MASKED && kind != RT_RES_SUBTRACTIVE) return RT_ERR_INVALID_ARGUMENT;
-  rt_status st = validate(desc, q, k, v, idx, o, rho, r);
+  rt_status st = validate(desc, q, k, v, idx, o, rho, r, true);
   if (st != RT_OK) return st;
   const rt_attn_desc& d = *desc;
   const int dpad = dpad_of(d.d);
@@ -301,7 +319,7 @@ rt_status rt_sparse_step_ex(const rt_attn_desc* desc, const void* q, const void*
                             int32_t step_distance, rt_ramp ramp, rt_epilogue epi, void* o, void* stream) {
   if (epi != RT_EPI_RESHAPED && epi != RT_EPI_NO_RHO && epi != RT_EPI_NO_R) return RT_ERR_INVALID_ARGUMENT;
   const bool use_rho = epi != RT_EPI_NO_RHO, use_r = epi != RT_EPI_NO_R;
-  rt_status st = validate(desc, q, k, v, idx, o, rho, r, use_rho, use_r);
+  rt_status st = validate(desc, q, k, v, idx, o, rho, r, false, use_rho, use_r);
   if (st != RT_OK) return st;
   if (!std::isfinite(lambda) || step_distance < 0) return RT_ERR_INVALID_ARGUMENT;
   double mul = 1.0, add = 0.0;

@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "attn_kernel.cuh"
+#include "layout.h"
 #include "rt.h"
 
 namespace rtb {
@@ -124,6 +125,11 @@ rt_status rt_permute_tokens(const rt_attn_desc* desc, const void* src, void* dst
   if (d.stride_b < 1 || d.stride_h < 1 || d.stride_l < d.d) return RT_ERR_INVALID_ARGUMENT;
   if (d.stride_b % 8 || d.stride_h % 8 || d.stride_l % 8) return RT_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) return RT_ERR_INVALID_ARGUMENT;
+  // every destination row is written by one thread group: rows must be disjoint,
+  // and the source must not be overwritten while it is read
+  if (!rtb::layout_rows_disjoint(d)) return RT_ERR_INVALID_ARGUMENT;
+  const long long span = rtb::layout_span_bytes(d, 2);
+  if (rtb::ranges_overlap(src, span, dst, span)) return RT_ERR_INVALID_ARGUMENT;
   unsigned int* status = nullptr;
   rt_status st = rtb::api_status_word(&status);
   if (st != RT_OK) return st;

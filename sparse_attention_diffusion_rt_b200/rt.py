@@ -189,6 +189,8 @@ def make_block_index(row_ptr: torch.Tensor, col_idx: torch.Tensor, Hm: int, nqb:
 def _desc(q: torch.Tensor, block: int, softmax_scale: float, r_dtype: torch.dtype) -> RtAttnDesc:
     if q.dim() != 4 or q.stride(3) != 1:
         raise ValueError("q/k/v/o/r must be [B, H, L, d] with d contiguous")
+    if r_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("r must be bf16 or fp32")
     B, H, L, d = q.shape
     sb, sh, sl, _ = q.stride()
     rd = RT_F32 if r_dtype == torch.float32 else RT_BF16
@@ -201,23 +203,46 @@ def _same_layout(ref: torch.Tensor, *ts):
             raise ValueError("q, k, v, o and r must share shape and strides")
 
 
+def _check_attn_tensors(q, k, v, o=None, rho=None, r=None, *, need_rho=True, need_r=True):
+    """The checks every attention entry point makes before anything launches:
+    q, k, v (and o) bf16 [B, H, L, d] with d contiguous and one shared layout,
+    r bf16 or fp32 in that layout, rho a contiguous fp32 [B, H, L] tensor.
+    The C side cannot see dtypes or allocation sizes (it writes B*H*L floats
+    of rho), so these are refused here with ValueError."""
+    for t in (q, k, v):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be bfloat16 tensors")
+    if q.dim() != 4 or q.stride(3) != 1:
+        raise ValueError("q/k/v/o/r must be [B, H, L, d] with d contiguous")
+    if o is not None and o.dtype != torch.bfloat16:
+        raise ValueError("o must be bfloat16")
+    if need_rho and rho is None:
+        raise ValueError("rho is required")
+    if need_r and r is None:
+        raise ValueError("r is required")
+    if r is not None and r.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("r must be bf16 or fp32")
+    if rho is not None:
+        B, H, L, _ = q.shape
+        if rho.dtype != torch.float32 or tuple(rho.shape) != (B, H, L) or not rho.is_contiguous():
+            raise ValueError("rho must be a contiguous fp32 [B, H, L] tensor")
+    _same_layout(q, k, v, *(t for t in (o, r) if t is not None))
+
+
 def rt_calibrate(q, k, v, index: BlockIndex, *, block: int, o=None, rho=None, r=None,
                  r_dtype=torch.bfloat16, softmax_scale: float = 0.0, residual: int = RT_RES_MASKED,
                  stream=None):
     """Calibration step: returns (O bf16, rho fp32 [B,H,L], R r_dtype).
     residual selects Re-ttention's R (default) or DiTFastAttn's O - O_sparse."""
     lib = load_library()
+    _check_attn_tensors(q, k, v, o, rho, r, need_rho=False, need_r=False)
+    if r is not None and r.dtype != r_dtype:
+        raise ValueError("r must have dtype r_dtype")
     _require_cuda(q, k, v, o, rho, r)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16:
-            raise ValueError("q, k, v must be bfloat16")
     B, H, L, d = q.shape
     o = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if o is None else o
     r = torch.empty_strided(q.shape, q.stride(), dtype=r_dtype, device=q.device) if r is None else r
     rho = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if rho is None else rho
-    if o.dtype != torch.bfloat16 or r.dtype != r_dtype or rho.dtype != torch.float32 or not rho.is_contiguous():
-        raise ValueError("o must be bf16, r must be r_dtype, rho fp32 contiguous [B, H, L]")
-    _same_layout(q, k, v, o, r)
     desc = _desc(q, block, softmax_scale, r_dtype)
     idx = index.as_c()
     _check(lib.rt_calibrate_ex(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
@@ -233,22 +258,9 @@ def rt_sparse_step(q, k, v, index: BlockIndex, rho, r, *, block: int, lam: float
     Re-ttention epilogue (default) or an ablation; rho may be None with
     RT_EPI_NO_RHO and r may be None with RT_EPI_NO_R."""
     lib = load_library()
+    _check_attn_tensors(q, k, v, o, rho, r, need_rho=epilogue != RT_EPI_NO_RHO, need_r=epilogue != RT_EPI_NO_R)
     _require_cuda(q, k, v, rho, r, o)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16:
-            raise ValueError("q, k, v must be bfloat16")
-    if rho is None and epilogue != RT_EPI_NO_RHO:
-        raise ValueError("rho is required unless epilogue is RT_EPI_NO_RHO")
-    if r is None and epilogue != RT_EPI_NO_R:
-        raise ValueError("r is required unless epilogue is RT_EPI_NO_R")
-    if r is not None and r.dtype not in (torch.bfloat16, torch.float32):
-        raise ValueError("r must be bf16 or fp32")
-    if rho is not None and (rho.dtype != torch.float32 or not rho.is_contiguous()):
-        raise ValueError("rho must be fp32 contiguous [B, H, L]")
     o = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if o is None else o
-    if o.dtype != torch.bfloat16:
-        raise ValueError("o must be bfloat16")
-    _same_layout(q, k, v, o, *(() if r is None else (r,)))
     desc = _desc(q, block, softmax_scale, torch.bfloat16 if r is None else r.dtype)
     idx = index.as_c()
     _check(lib.rt_sparse_step_ex(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(idx),
@@ -294,8 +306,8 @@ def rt_schedule_step(q, k, v, index: BlockIndex, t: int, *, block: int, period: 
     """Step t of a denoising schedule: a calibration into (o, rho, r) when
     t % period == 0, else a sparse step reading (rho, r) into o."""
     lib = load_library()
+    _check_attn_tensors(q, k, v, o, rho, r)
     _require_cuda(q, k, v, o, rho, r)
-    _same_layout(q, k, v, o, r)
     desc = _desc(q, block, softmax_scale, r.dtype)
     sched = _schedule(period, lam, ramp, epilogue, residual)
     idx = index.as_c()
@@ -320,8 +332,10 @@ class CycleGraph:
         if period < 1 or len(outs) != period:
             raise ValueError("one (q, k, v) and one output per step of the cycle")
         for (q, k, v), o in zip(steps, outs):
+            _check_attn_tensors(q, k, v, o, rho, r)
+            _same_layout(steps[0][0], q)
+        for (q, k, v), o in zip(steps, outs):
             _require_cuda(q, k, v, o)
-            _same_layout(steps[0][0], q, k, v, o, r)
         _require_cuda(rho, r)
         if stream is None or stream.cuda_stream == 0:
             raise ValueError("capture needs a created stream")

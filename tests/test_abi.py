@@ -78,7 +78,8 @@ def test_host_validation_without_gpu(lib):
     assert lib.rt_calibrate(None, vp(16), vp(16), vp(16), None, vp(16), vp(16), vp(16), None) == rt.RT_ERR_INVALID_ARGUMENT
     desc = rt.RtAttnDesc(1, 1, 128, 64, 128, 8192, 8192, 64, 0.0, 0)
     idx = rt.RtBlockIndex(1, 1, 1, 1, 4096, 4096)
-    args = (vp(4096), vp(4096), vp(4096), ctypes.byref(idx), vp(4096), vp(4096), vp(4096), None)
+    # q, k, v, idx, o, rho, r at disjoint (never dereferenced) addresses
+    args = (vp(1 << 20), vp(2 << 20), vp(3 << 20), ctypes.byref(idx), vp(4 << 20), vp(5 << 20), vp(6 << 20), None)
     bad = rt.RtAttnDesc(1, 1, 128, 20, 128, 8192, 8192, 64, 0.0, 0)          # d % 8 != 0
     assert lib.rt_calibrate(ctypes.byref(bad), *args) == rt.RT_ERR_UNSUPPORTED
     bad = rt.RtAttnDesc(1, 1, 128, 64, 32, 8192, 8192, 64, 0.0, 0)           # block 32
@@ -131,6 +132,78 @@ def test_host_validation_without_gpu(lib):
         rt.RT_ERR_INVALID_ARGUMENT
     assert lib.rt_build_block_index(vp(16), 1, 0, 1, vp(16), vp(16), 1, ctypes.byref(nnz), None) == \
         rt.RT_ERR_INVALID_ARGUMENT
+
+
+def test_host_validation_rejects_aliasing_layouts_and_overlaps(lib):
+    """Layouts whose (b, h, l) rows share elements, and outputs that overlap an
+    input or another output, are refused before any CUDA call."""
+    vp = ctypes.c_void_p
+    idx = rt.RtBlockIndex(1, 1, 1, 1, 4096, 4096)
+    q, k, v, o, rho, r = (vp(i << 20) for i in range(1, 7))
+    # two heads on the same rows (stride_h < L * stride_l, and not a [B, L, H, d] interleave)
+    alias = rt.RtAttnDesc(1, 2, 128, 64, 128, 16384, 64, 64, 0.0, 0)
+    assert lib.rt_calibrate(ctypes.byref(alias), q, k, v, ctypes.byref(idx), o, rho, r, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT
+    alias_b = rt.RtAttnDesc(2, 2, 128, 64, 128, 8192, 8192, 64, 0.0, 0)     # batches alias the heads
+    assert lib.rt_calibrate(ctypes.byref(alias_b), q, k, v, ctypes.byref(idx), o, rho, r, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_permute_tokens(ctypes.byref(alias), q, k, vp(64), 0, None) == rt.RT_ERR_INVALID_ARGUMENT
+    desc = rt.RtAttnDesc(1, 1, 128, 64, 128, 8192, 8192, 64, 0.0, 0)       # 16 KiB per tensor
+    near = lambda p, off: vp(p.value + off)
+    bad_calls = [
+        (near(q, 4096), rho, r),        # o overlaps q
+        (o, rho, near(k, 1024)),        # r overlaps k (the calibration writes r)
+        (o, near(v, 16), r),            # rho overlaps v
+        (o, rho, near(o, 8192)),        # r overlaps o
+        (o, near(r, 64), r),            # rho overlaps r
+    ]
+    for oo, rr, res in bad_calls:
+        assert lib.rt_calibrate(ctypes.byref(desc), q, k, v, ctypes.byref(idx), oo, rr, res, None) == \
+            rt.RT_ERR_INVALID_ARGUMENT
+    lam = ctypes.c_float(0.04)
+    assert lib.rt_sparse_step(ctypes.byref(desc), q, k, v, ctypes.byref(idx), rho, near(o, 32), lam, 1, 0, o,
+                              None) == rt.RT_ERR_INVALID_ARGUMENT                 # o overlaps r
+    span = 16384
+    assert lib.rt_permute_tokens(ctypes.byref(desc), q, near(q, span - 16), vp(64), 0, None) == \
+        rt.RT_ERR_INVALID_ARGUMENT                                            # dst overlaps src
+    # a [B, L, H, d] interleave has disjoint rows: accepted by validation (the
+    # call then needs a device, so without one it fails later, not as invalid)
+    blhd = rt.RtAttnDesc(1, 2, 128, 64, 128, 16384, 64, 128, 0.0, 0)
+    assert lib.rt_calibrate(ctypes.byref(blhd), q, k, v, ctypes.byref(idx), o, rho, r, None) != \
+        rt.RT_ERR_INVALID_ARGUMENT
+
+
+def test_binding_checks_dtypes_and_layouts_before_launch(lib):
+    """Every entry point of the binding refuses a wrong dtype or layout of
+    rho, r or o with ValueError before anything is launched (these checks do
+    not need a device)."""
+    import torch
+    q = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    good_rho = torch.zeros(1, 2, 256, dtype=torch.float32)
+    good_r = torch.zeros_like(q)
+    bad = {
+        "bf16 rho": dict(rho=good_rho.to(torch.bfloat16), r=good_r),
+        "non-contiguous rho": dict(rho=torch.zeros(1, 2, 512, dtype=torch.float32)[:, :, ::2], r=good_r),
+        "short rho": dict(rho=torch.zeros(1, 2, 255, dtype=torch.float32), r=good_r),
+        "fp16 r": dict(rho=good_rho, r=good_r.to(torch.float16)),
+        "r in another layout": dict(rho=good_rho, r=good_r.transpose(1, 2).contiguous().transpose(1, 2)),
+    }
+    idx = rt.BlockIndex(torch.zeros(3, dtype=torch.int32), torch.zeros(0, dtype=torch.int32), 1, 2, 2, 0)
+    for what, kw in bad.items():
+        with pytest.raises(ValueError):
+            rt.rt_schedule_step(q, q, q, idx, 0, block=128, period=5, o=torch.empty_like(q), **kw)
+        with pytest.raises(ValueError):
+            rt.rt_schedule_step(q, q, q, idx, 2, block=128, period=5, o=torch.empty_like(q), **kw)
+        with pytest.raises(ValueError):
+            rt.rt_sparse_step(q, q, q, idx, kw["rho"], kw["r"], block=128)
+        with pytest.raises(ValueError):
+            rt.CycleGraph([(q, q, q)] * 2, idx, block=128, outs=[torch.empty_like(q)] * 2, stream=None, **kw)
+        with pytest.raises(ValueError):
+            rt.rt_calibrate(q, q, q, idx, block=128, rho=kw["rho"], r=kw["r"], r_dtype=kw["r"].dtype)
+    with pytest.raises(ValueError):
+        rt.rt_schedule_step(q, q, q, idx, 0, block=128, period=5, o=q.float(), rho=good_rho, r=good_r)
+    with pytest.raises(ValueError):
+        rt.rt_calibrate(q.float(), q, q, idx, block=128)
 
 
 def test_binding_refuses_without_cuda(lib):
