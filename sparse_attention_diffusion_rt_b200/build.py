@@ -55,7 +55,11 @@ def _stale(target: str, deps) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile (if stale) and return the path of the shared library."""
+    """Compile (if stale) and return the path of the shared library.
+    RT_NVTX=1 in the environment compiles NVTX ranges around the C-ABI entry
+    points (off by default; a change of the switch needs force=True)."""
+    if os.environ.get("RT_NVTX") == "1":
+        extra_flags = tuple(extra_flags) + ("-DRT_NVTX",)
     deps = _deps() + [os.path.abspath(__file__)]
     if not force and not _stale(LIB, deps):
         return LIB

@@ -12,6 +12,7 @@
 
 #include "attn_launch.h"
 #include "layout.h"
+#include "nvtx_range.h"
 #include "rt.h"
 
 namespace rtb {
@@ -262,6 +263,7 @@ rt_status rt_set_wait_limit_ns(uint64_t limit_ns) {
 rt_status rt_build_block_index(const uint8_t* d_mask, int32_t Hm, int32_t nqb, int32_t nkb,
                                int32_t* d_row_ptr, int32_t* d_col_idx, int64_t col_capacity,
                                int64_t* h_nnz, void* stream) {
+  RT_RANGE("rt_build_block_index");
   if (!d_mask || !d_row_ptr || !h_nnz || Hm < 1 || nqb < 1 || nkb < 1 || col_capacity < 0)
     return RT_ERR_INVALID_ARGUMENT;
   if (col_capacity > 0 && !d_col_idx) return RT_ERR_INVALID_ARGUMENT;
@@ -288,6 +290,7 @@ rt_status rt_calibrate(const rt_attn_desc* desc, const void* q, const void* k, c
 rt_status rt_calibrate_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                           const rt_block_index* idx, void* o, float* rho, void* r, rt_residual kind,
                           void* stream) {
+  RT_RANGE("rt_calibrate_ex");
   if (kind != RT_RES_MASKED && kind != RT_RES_SUBTRACTIVE) return RT_ERR_INVALID_ARGUMENT;
   rt_status st = validate(desc, q, k, v, idx, o, rho, r, true);
   if (st != RT_OK) return st;
@@ -317,6 +320,7 @@ rt_status rt_sparse_step(const rt_attn_desc* desc, const void* q, const void* k,
 rt_status rt_sparse_step_ex(const rt_attn_desc* desc, const void* q, const void* k, const void* v,
                             const rt_block_index* idx, const float* rho, const void* r, float lambda,
                             int32_t step_distance, rt_ramp ramp, rt_epilogue epi, void* o, void* stream) {
+  RT_RANGE("rt_sparse_step_ex");
   if (epi != RT_EPI_RESHAPED && epi != RT_EPI_NO_RHO && epi != RT_EPI_NO_R) return RT_ERR_INVALID_ARGUMENT;
   const bool use_rho = epi != RT_EPI_NO_RHO, use_r = epi != RT_EPI_NO_R;
   rt_status st = validate(desc, q, k, v, idx, o, rho, r, false, use_rho, use_r);

@@ -7,6 +7,7 @@
 
 #include <new>
 
+#include "nvtx_range.h"
 #include "rt.h"
 
 namespace rtb {
@@ -22,6 +23,7 @@ extern "C" {
 rt_status rt_schedule_step(const rt_attn_desc* desc, const rt_schedule* sched, int32_t t, const void* q,
                            const void* k, const void* v, const rt_block_index* idx, void* o, float* rho, void* r,
                            void* stream) {
+  RT_RANGE("rt_schedule_step");
   if (!sched || sched->period < 1 || t < 0) return RT_ERR_INVALID_ARGUMENT;
   const int32_t kdist = t % sched->period;
   if (kdist == 0) return rt_calibrate_ex(desc, q, k, v, idx, o, rho, r, sched->residual, stream);
@@ -32,6 +34,7 @@ rt_status rt_schedule_step(const rt_attn_desc* desc, const rt_schedule* sched, i
 rt_status rt_schedule_capture(const rt_attn_desc* desc, const rt_schedule* sched, const void* const* q,
                               const void* const* k, const void* const* v, const rt_block_index* idx,
                               void* const* o, float* rho, void* r, void* stream, rt_cycle_graph** graph) {
+  RT_RANGE("rt_schedule_capture");
   if (!graph) return RT_ERR_INVALID_ARGUMENT;
   *graph = nullptr;
   if (!sched || sched->period < 1 || !q || !k || !v || !o || !stream) return RT_ERR_INVALID_ARGUMENT;
@@ -61,6 +64,7 @@ rt_status rt_schedule_capture(const rt_attn_desc* desc, const rt_schedule* sched
 }
 
 rt_status rt_cycle_graph_launch(rt_cycle_graph* graph, void* stream) {
+  RT_RANGE("rt_cycle_graph_launch");
   if (!graph) return RT_ERR_INVALID_ARGUMENT;
   cudaError_t e = cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RT_OK : rtb::api_cuda_fail(e, "cudaGraphLaunch");

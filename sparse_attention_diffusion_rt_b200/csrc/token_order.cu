@@ -20,6 +20,7 @@
 
 #include "attn_kernel.cuh"
 #include "layout.h"
+#include "nvtx_range.h"
 #include "rt.h"
 
 namespace rtb {
@@ -118,6 +119,7 @@ rt_status rt_hilbert_token_order(int32_t n_text, int32_t F, int32_t Y, int32_t X
 
 rt_status rt_permute_tokens(const rt_attn_desc* desc, const void* src, void* dst, const int32_t* d_perm,
                             int32_t inverse, void* stream) {
+  RT_RANGE("rt_permute_tokens");
   if (!desc || !src || !dst || !d_perm || (inverse != 0 && inverse != 1) || src == dst)
     return RT_ERR_INVALID_ARGUMENT;
   const rt_attn_desc& d = *desc;

@@ -8,10 +8,13 @@ makes.
 Recipe
 ------
 * Q, K, V ~ N(0, 1) in float32, rounded to bf16, layout [B, H, L, d]
-  contiguous.  Drawn from ``torch.Generator(device).manual_seed(seed)`` in the
-  order Q, K, V.
-* Next denoising step: X_{s+1} = bf16(X_s + 0.05 N(0, 1)), drawn from a
-  generator seeded with 1000 * seed + s, again in the order Q, K, V.
+  contiguous.  Each (batch, head) slab is drawn from its own generator,
+  ``torch.Generator(device).manual_seed(stream_seed(seed, 0, b, h))``, in the
+  order Q, K, V, so that a rank that owns a range of heads draws exactly those
+  heads' values and nothing else.
+* Next denoising step: X_{s+1} = bf16(X_s + 0.05 N(0, 1)), the noise of slab
+  (b, h) drawn from a generator seeded with stream_seed(seed, s + 1, b, h),
+  again in the order Q, K, V.
 * Text tokens (MM-DiT "unified self-attention", Re-ttention OpenReview reply
   to Q5) come first in the sequence, visual tokens follow in row-major
   (frame, y, x) order.
@@ -154,29 +157,54 @@ def _randn(shape, gen, device):
     return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
 
 
-def initial_qkv(w: Workload, device="cpu"):
-    """Step-0 Q, K, V: bf16 [B, H, L, d] from N(0, 1) with the workload's seed."""
-    gen = torch.Generator(device=device).manual_seed(w.seed)
-    shape = (w.B, w.H, w.L, w.d)
-    return tuple(_randn(shape, gen, device).to(torch.bfloat16) for _ in range(3))
+def stream_seed(seed: int, step: int, b: int, h: int) -> int:
+    """Seed of the generator that draws slab (b, h) at denoising step `step`
+    (0 = the initial values, s + 1 = the drift from step s to s + 1)."""
+    return ((seed * 1009 + step) * 65537 + b) * 65537 + h
 
 
-def drift_qkv(w: Workload, qkv, s: int):
-    """Step s+1 from step s: X + 0.05 N(0, 1), rounded to bf16."""
-    device = qkv[0].device
-    gen = torch.Generator(device=device).manual_seed(1000 * w.seed + s)
-    out = []
-    for x in qkv:
-        n = _randn(x.shape, gen, device)
-        out.append((x.float() + 0.05 * n).to(torch.bfloat16))
+def _head_range(w: Workload, heads):
+    h0, h1 = (0, w.H) if heads is None else heads
+    if not 0 <= h0 < h1 <= w.H:
+        raise ValueError(f"head range {heads} outside 0..{w.H}")
+    return h0, h1
+
+
+def initial_qkv(w: Workload, device="cpu", heads=None):
+    """Step-0 Q, K, V: bf16 [B, H, L, d] from N(0, 1).  heads = (h0, h1)
+    draws only heads h0..h1-1 (a [B, h1-h0, L, d] slice with the values the
+    whole problem has there)."""
+    h0, h1 = _head_range(w, heads)
+    out = [torch.empty((w.B, h1 - h0, w.L, w.d), dtype=torch.bfloat16, device=device) for _ in range(3)]
+    for b in range(w.B):
+        for h in range(h0, h1):
+            gen = torch.Generator(device=device).manual_seed(stream_seed(w.seed, 0, b, h))
+            for x in out:
+                x[b, h - h0] = _randn((w.L, w.d), gen, device).to(torch.bfloat16)
     return tuple(out)
 
 
-def qkv_steps(w: Workload, n_steps: int, device="cpu"):
-    """List of (Q, K, V) for steps 0 .. n_steps-1 of one calibration cycle."""
-    steps = [initial_qkv(w, device)]
+def drift_qkv(w: Workload, qkv, s: int, heads=None):
+    """Step s+1 from step s: X + 0.05 N(0, 1), rounded to bf16.  heads as in
+    initial_qkv (qkv then holds that head range)."""
+    h0, h1 = _head_range(w, heads)
+    device = qkv[0].device
+    out = [torch.empty_like(x) for x in qkv]
+    for b in range(w.B):
+        for h in range(h0, h1):
+            gen = torch.Generator(device=device).manual_seed(stream_seed(w.seed, s + 1, b, h))
+            for x, y in zip(qkv, out):
+                n = _randn((w.L, w.d), gen, device)
+                y[b, h - h0] = (x[b, h - h0].float() + 0.05 * n).to(torch.bfloat16)
+    return tuple(out)
+
+
+def qkv_steps(w: Workload, n_steps: int, device="cpu", heads=None):
+    """List of (Q, K, V) for steps 0 .. n_steps-1 of one calibration cycle
+    (heads = (h0, h1) for one rank's head range)."""
+    steps = [initial_qkv(w, device, heads)]
     for s in range(n_steps - 1):
-        steps.append(drift_qkv(w, steps[-1], s))
+        steps.append(drift_qkv(w, steps[-1], s, heads))
     return steps
 
 

@@ -17,15 +17,52 @@ def test_executed_flops_counts_qk_and_pv_of_every_executed_block():
 
 
 def test_profiled_traffic_only_for_the_current_source(tmp_path, monkeypatch):
+    import json
     (tmp_path / "profiles").mkdir()
-    (tmp_path / "profiles" / "calibrate_w.md").write_text(
-        "# summary\n\nsource_hash: 0123abcd\ndram_bytes_per_launch: 123456789\n")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"calibrate": {"w": {"source_hash": "0123abcd", "dram_bytes_per_launch": 123456789}}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0123abcd")
     assert bench.profiled_traffic("calibrate", "w") == 123456789.0
-    assert bench.profiled_traffic("sparse_step", "w") is None          # no summary
+    assert bench.profiled_traffic("sparse_step", "w") is None          # no capture of that kernel
+    assert bench.profiled_traffic("calibrate", "other") is None        # nor of that workload
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "ffff0000")
     assert bench.profiled_traffic("calibrate", "w") is None            # kernel changed since
+
+
+def test_committed_traffic_records_are_well_formed():
+    import json
+    import os
+    path = os.path.join(bench.ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return
+    table = json.load(open(path))
+    for kernel, per_w in table.items():
+        assert kernel in ("calibrate", "sparse_step")
+        for wname, rec in per_w.items():
+            assert wname in inputs.WORKLOADS or wname.rsplit("-h", 1)[0] in inputs.WORKLOADS
+            assert len(rec["source_hash"]) == 16 and rec["dram_bytes_per_launch"] > 0
+            assert "command" in rec
+
+
+def test_compulsory_bytes_and_l2_rotation():
+    w = inputs.WORKLOADS["pixart"]
+    elems = 2 * 16 * 4096 * 72
+    total, r_rho = bench.compulsory_bytes(w)
+    assert r_rho == elems * 2 + 2 * 16 * 4096 * 4                      # R bf16 + rho fp32
+    assert total == 4 * elems * 2 + r_rho                              # Q, K, V in, O out, plus R and rho
+    assert bench.compulsory_bytes(w, 4)[1] == elems * 4 + 2 * 16 * 4096 * 4
+    # rotated sets always exceed L2 twice over; a call larger than that needs one set
+    for per_call in (1, 10 ** 6, 90 * 10 ** 6, 3 * 10 ** 9):
+        n = bench.sets_for_l2(per_call)
+        assert n * per_call >= 2 * bench.L2_BYTES and (n == 1 or (n - 1) * per_call < 2 * bench.L2_BYTES)
+
+
+def test_peak_follows_the_power_regime():
+    peaks = {"bf16_tflops": 1646.8, "bf16_tflops_sustained": 1398.0, "hbm_gbs": 6551.0, "source": "measured"}
+    assert bench.peak_for({"reasons": ["sw_power_cap"]}, peaks)[0] == 1398.0
+    assert bench.peak_for({"reasons": []}, peaks)[0] == 1646.8
+    assert bench.peak_for({"reasons": ["hw_slowdown"]}, peaks)[0] == 1646.8
 
 
 def test_kernel_source_hash_covers_every_kernel_file():

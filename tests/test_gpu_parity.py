@@ -387,6 +387,57 @@ def _sample_rows(L, block, rng, n_mid=6):
     return np.array(sorted(set(rows)))
 
 
+@pytest.mark.parametrize("name", ["pixart", "hunyuan"])
+def test_workload_schedule_full_tensors(name):
+    """The configuration's own cycle, 1 calibration + 4 sparse steps at
+    k = 1..4 on inputs that drift from step to step, through the schedule
+    driver, against the oracle's schedule on every element."""
+    w = inputs.WORKLOADS[name]
+    period = 1 + w.n_sparse_steps
+    steps = inputs.qkv_steps(w, period, device=DEV)
+    mask = inputs.block_mask(w)
+    idx = _index(mask)
+    rho = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=DEV)
+    r = torch.empty_like(steps[0][0])
+    outs = [rt.rt_schedule_step(q, k, v, idx, t, block=w.block, period=period, lam=w.lam, o=torch.empty_like(q),
+                                rho=rho, r=r) for t, (q, k, v) in enumerate(steps)]
+    torch.cuda.synchronize()
+    _ok()
+    want = ref.schedule_ref([tuple(f64(x) for x in s) for s in steps], mask, w.block, period, w.lam)
+    for t, (o, wt) in enumerate(zip(outs, want)):
+        check_out(f64(o), wt, f"{name} schedule step {t} (k = {t})")
+
+
+def test_cogvideox_cycle_sampled_rows_k1_and_k9():
+    """CogVideoX-like cycle, 1 calibration + 9 sparse steps through the
+    schedule driver at full size; sampled rows of the calibration and of the
+    sparse steps at k = 1 and k = 9 against the oracle."""
+    w = inputs.WORKLOADS["cogvideox"]
+    period = 1 + w.n_sparse_steps
+    steps = inputs.qkv_steps(w, period, device=DEV)
+    mask = inputs.block_mask(w)
+    idx = _index(mask)
+    rho = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=DEV)
+    r = torch.empty_like(steps[0][0])
+    outs = [rt.rt_schedule_step(q, k, v, idx, t, block=w.block, period=period, lam=w.lam, o=torch.empty_like(q),
+                                rho=rho, r=r) for t, (q, k, v) in enumerate(steps)]
+    torch.cuda.synchronize()
+    _ok()
+    rng = np.random.default_rng(33)
+    for b, h in [(0, 0), (0, w.H - 1), (0, int(rng.integers(w.H)))]:
+        rows = _sample_rows(w.L, w.block, rng)
+        O, RHO, R = ref.calibrate_rows_ref(*(f64(x[b, h]) for x in steps[0]), mask[0], w.block, rows)
+        check_out(f64(outs[0][b, h, rows]), O, f"cogvideox calibrate O (h{h})")
+        check_out(f64(r[b, h, rows]), R, f"cogvideox calibrate R (h{h})")
+        check_rho(f64(rho[b, h, rows]), RHO, f"cogvideox rho (h{h})")
+        for t in (1, w.n_sparse_steps):
+            O2 = ref.sparse_step_rows_ref(*(f64(x[b, h]) for x in steps[t]), mask[0], w.block, rows, RHO, R,
+                                          w.lam, t)
+            check_out(f64(outs[t][b, h, rows]), O2, f"cogvideox sparse O at k = {t} (h{h})")
+    del steps, outs
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("name", ["cogvideox", "longvideo-3.1", "longvideo-6.25", "longvideo-12.5", "longvideo-25"])
 def test_full_size_sampled_rows(name):
     w = inputs.WORKLOADS[name]
@@ -572,3 +623,11 @@ def test_head_shards_reproduce_the_whole_problem(per_head_mask, d):
         _ok()
         assert torch.equal(o_s, sl(o)) and torch.equal(rho_s, sl(rho)) and torch.equal(r_s, sl(r))
         assert torch.equal(o2_s, sl(o2))
+        # and each shard against the oracle on its own heads
+        mask_s = shard.shard_mask(mask, h0, h1)
+        O, RHO, R = ref.calibrate_ref(f64(sl(q)), f64(sl(k)), f64(sl(v)), mask_s, blk)
+        check_out(f64(o_s), O, f"shard {rank} calibrate O")
+        check_out(f64(r_s), R, f"shard {rank} calibrate R")
+        check_rho(f64(rho_s), RHO, f"shard {rank} rho")
+        O2 = ref.sparse_step_ref(f64(sl(q2)), f64(sl(k2)), f64(sl(v2)), mask_s, blk, RHO, R, 0.04, 2)
+        check_out(f64(o2_s), O2, f"shard {rank} sparse O")

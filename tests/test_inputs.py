@@ -53,3 +53,23 @@ def test_seeded_inputs_reproducible_and_drift():
     dq = (a[1][0].float() - a[0][0].float())
     assert 0.03 < dq.std().item() < 0.07                   # 0.05 N(0,1) drift, bf16-rounded
     assert abs(a[0][0].float().std().item() - 1.0) < 0.1
+
+
+def test_head_range_draws_the_whole_problems_values():
+    """A rank that owns heads h0..h1-1 draws exactly the whole problem's values
+    there, at every step, without drawing the other heads."""
+    w = inputs.Workload("t", 2, 5, 130, 16, 64, kept=1, n_sparse_steps=2, seed=3)
+    whole = inputs.qkv_steps(w, 3)
+    for h0, h1 in ((0, 2), (2, 5), (4, 5)):
+        part = inputs.qkv_steps(w, 3, heads=(h0, h1))
+        for sw, sp in zip(whole, part):
+            for x, y in zip(sw, sp):
+                assert y.shape == (2, h1 - h0, 130, 16)
+                assert torch.equal(x[:, h0:h1], y)
+    # distinct slabs are distinct draws
+    q = whole[0][0].float()
+    assert not torch.equal(q[0, 0], q[0, 1]) and not torch.equal(q[0, 0], q[1, 0])
+    assert not torch.equal(whole[0][0], whole[0][1])
+    import pytest
+    with pytest.raises(ValueError):
+        inputs.initial_qkv(w, heads=(3, 6))

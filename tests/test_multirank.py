@@ -119,7 +119,18 @@ def _shard_rank_main(rank, world, port, H, out):
         counts = torch.zeros(H, dtype=torch.int64)
         counts[h0:h1] = 1
         torch.distributed.all_reduce(counts)                   # every head owned by exactly one rank
-        out[rank] = counts.tolist()
+        # each rank draws only its own heads' inputs; together they are the whole problem's
+        from sparse_attention_diffusion_rt_b200 import inputs
+        w = inputs.Workload("t", 2, H, 70, 16, 64, kept=1, n_sparse_steps=1, seed=5)
+        mine = inputs.qkv_steps(w, 2, heads=(h0, h1))
+        same = True
+        for s in range(2):
+            for x in range(3):
+                full = torch.zeros((w.B, H, w.L, w.d), dtype=torch.float32)
+                full[:, h0:h1] = mine[s][x].float()
+                torch.distributed.all_reduce(full)             # disjoint head ranges: the sum is the union
+                same &= torch.equal(full.to(torch.bfloat16), inputs.qkv_steps(w, 2)[s][x])
+        out[rank] = (counts.tolist(), bool(same))
     finally:
         torch.distributed.destroy_process_group()
 
@@ -141,4 +152,5 @@ def test_head_sharding_gloo_every_head_once():
                 p.join()
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
         res = dict(out)
-    assert res[0] == res[1] == [1] * H
+    assert res[0][0] == res[1][0] == [1] * H
+    assert res[0][1] and res[1][1]
