@@ -98,7 +98,7 @@ cudaError_t launch_sparse_impl(const TmaSet& tm, const AttnParams& p, cudaStream
   }
   const long long ntiles = static_cast<long long>(p.B) * p.H * p.nqb;
   const int grid = static_cast<int>(ntiles < sm_count[dev & 63] ? ntiles : sm_count[dev & 63]);
-  kern<<<grid, kThreads, smem, s>>>(tm, p, static_cast<int>(ntiles));
+  kern<<<grid, kSpThreads, smem, s>>>(tm, p, static_cast<int>(ntiles));
   return cudaGetLastError();
 }
 

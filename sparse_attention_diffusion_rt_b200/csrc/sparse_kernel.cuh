@@ -6,14 +6,22 @@
 // plus the cached residual of the masked tokens; reply to Pwod's W1: ramp-up).
 //
 // One CTA per SM walks the (batch, head, query block) tiles tile = blockIdx.x
-// + i * gridDim.x, query block fastest (see sp_decode).  Roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread t owns tile row t (TMEM lane t)
-//   warp 4     producer: lane 0 validates each tile's CSR row and loads Q
+// + i * gridDim.x, query block fastest (see sp_decode).  Roles (320 threads):
+//   warps 0-3  softmax; thread t owns tile row t (TMEM lane t).  At the end of
+//              a tile it hands the row sum l to the epilogue (through a TMEM
+//              column) and goes straight on to the next tile.
+//   warps 4-7  epilogue; thread 128 + t owns row t.  It drains the tile's O from
+//              TMEM as soon as the last PV lands (releasing the accumulator
+//              for the next tile's first PV), then applies rho_hat / l, adds
+//              the residual tile and stores the bf16 result through a
+//              shared-memory staging tile and a TMA store, while the softmax
+//              warps already work on the next tile.
+//   warp 8     producer: lane 0 validates each tile's CSR row and loads Q
 //              (one buffer, free again once Q is in TMEM), the K tiles of the
 //              kept blocks and the residual tile; lane 1 loads the V tiles.  K
 //              and V have their own NST-stage rings, released after QK^T and
 //              after PV.
-//   warp 5     lane 0 issues the tcgen05 MMAs: it copies each tile's Q into
+//   warp 9     lane 0 issues the tcgen05 MMAs: it copies each tile's Q into
 //              TMEM (tcgen05.cp), then S = Q K^T into one of two TMEM logit
 //              buffers with Q read from TMEM, O += P V with P read from TMEM,
 //              so only K and V are read from shared memory.  The softmax
@@ -21,16 +29,17 @@
 //              then QK^T(j+2) into the same buffer: MMAs of one thread run in
 //              issue order, so the logits are never overwritten early and the
 //              tensor pipe always has the next logits queued.
-// Tile metadata flows through a 2-slot ring (ti_*).  Every per-block barrier
-// phase is indexed by a block counter that runs across tiles, so the MMA warp
-// starts the next tile's QK^T while the softmax warps finish the previous
-// tile's epilogue; the output leaves through a shared-memory staging tile and
-// a TMA store that is only waited for when its staging slot comes round again.
+// Tile metadata flows through a 2-slot ring (ti_*), the epilogue's share of it
+// (kept-block count, row sums) through a second 2-slot ring (epi_*).  Every
+// per-block barrier phase is indexed by a block counter that runs across
+// tiles, so the MMA warp starts the next tile's QK^T while the last PV of the
+// previous one runs.
 //
 // TMEM columns: S0/S1 [0,256) fp32 logits, each overwritten in place by its
 // bf16 probabilities P (64 columns of the 128), Q [256, 256+DPAD/2) as bf16
-// pairs, O [384, 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT
-// and every role drains what it has in flight before TMEM is freed.
+// pairs, the row sums of the two epilogue slots at 376 and 377, O [384,
+// 384+DPAD).  All waits are bounded; a timeout records RT_ERR_TIMEOUT and
+// every role drains what it has in flight before TMEM is freed.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -63,9 +72,28 @@ struct SpCfg {
   static constexpr int SMEM = OFF_OST + OSTG * TILE_BYTES + 1024;   // + alignment slack
   static_assert(NST >= 2, "at least two K/V stages");
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static constexpr uint32_t T_S = 0, T_Q = 256, T_O = 384;   // S_b (and P_b over it) at 128b, Q, O
-  static_assert(T_Q + DPAD / 2 <= T_O, "Q (bf16 pairs) fits below O");
+  static constexpr uint32_t T_S = 0, T_Q = 256, T_L = 376, T_O = 384;   // S_b (P_b over it), Q, l, O
+  static_assert(T_Q + DPAD / 2 <= T_L && T_L + 2 <= T_O, "Q (bf16 pairs) and the row sums fit below O");
 };
+
+// Roles of the sparse-step kernel: three warpgroups.  Each sub-partition of
+// the SM holds one warp of each, so the launch gives every thread 168
+// registers (3 x 32 x 168 of a sub-partition's 16384); the warpgroups then
+// rebalance: the softmax holds a 128-logit row in registers and takes 240, the
+// epilogue a whole O row and takes 176, the producer / MMA warpgroup gives
+// back down to 88.  128 x (240 + 176 + 88) = 64512 = 384 x 168: the .inc of
+// the first two exactly use what the .dec of the third returns.
+constexpr int kSpThreads = 384;
+constexpr int kSpEpiThread0 = 128;     // warps 4-7: epilogue
+constexpr int kSpProducerWarp = 8;
+constexpr int kSpMmaWarp = 9;          // warps 10-11 idle
+constexpr uint32_t kSpRegsLaunch = 168, kSpRegsSoftmax = 240, kSpRegsEpilogue = 176, kSpRegsOther = 88;
+static_assert(kSpRegsLaunch * kSpThreads <= 65536 && 3 * 32 * kSpRegsLaunch <= 16384,
+              "launch registers fit the register file and each sub-partition");
+static_assert(32 * (kSpRegsSoftmax + kSpRegsEpilogue + kSpRegsOther) <= 16384,
+              "after the split, one warp of each warpgroup still fits a sub-partition");
+static_assert(128 * (kSpRegsSoftmax + kSpRegsEpilogue + kSpRegsOther) <= kSpThreads * kSpRegsLaunch,
+              "the warpgroups' shares fit the pool the CTA was launched with");
 
 struct SpTile {
   int b, h, qb, n, start, bad;
@@ -80,8 +108,10 @@ struct SpCtrl {
   uint64_t r_full, r_empty;
   uint64_t ti_full[2], ti_empty[2];
   uint64_t stg_ready, stg_full;
+  uint64_t o_free, epi_full[2], epi_empty[2];
   uint64_t drain;
   SpTile ti[2];
+  int epi_n[2], epi_bad[2];   // the epilogue's share of a tile's metadata
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -285,6 +315,8 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
       const uint32_t g0 = g;
       for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_qk(g0 + i);
       for (int j = 0; ok && j < n; ++j) {
+        // the first PV restarts O: the epilogue must have drained the previous tile's O
+        if (j == 0 && qi >= 1 && !sp_wait(&ctl.o_free, (qi - 1) & 1, ctl, p)) { ok = false; break; }
         ok = issue_pv(g0 + j, j == 0);
         if (ok && j + 2 < n) ok = issue_qk(g0 + j + 2);
       }
@@ -301,20 +333,18 @@ __device__ __forceinline__ void sp_mma(const AttnParams& p, SpCtrl& ctl, uint8_t
   }
 }
 
-// ------------------------------------------------------------------ softmax + epilogue
+// ------------------------------------------------------------------ softmax
 template <int DPAD>
-__device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p, SpCtrl& ctl, uint8_t* base,
-                                           uint32_t tmem, int ntiles) {
+__device__ __forceinline__ void sp_softmax(const AttnParams& p, SpCtrl& ctl, uint32_t tmem, int ntiles) {
   using C = SpCfg<DPAD>;
   const int t = threadIdx.x;
   const int warp = t >> 5;
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_base + C::T_S;
   const uint32_t tO = tmem + lane_base + C::T_O;
-  uint8_t* sR = base + C::OFF_R;
-  uint8_t* sOst = base + C::OFF_OST;
+  const uint32_t tL = tmem + lane_base + C::T_L;
   const float sl2 = p.scale_log2;
-  uint32_t g = 0, oi = 0, ri = 0, si = 0;
+  uint32_t g = 0;
   bool ok = true;
   int it = 0;
   for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
@@ -323,12 +353,8 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
     if (!ok) break;
     const SpTile ti = ctl.ti[slot];
     mbar_arrive(&ctl.ti_empty[slot]);
-    if (ti.bad) continue;
-    const int grow = ti.qb * 128 + t;
-    const size_t rho_idx = (static_cast<size_t>(ti.b) * p.H + ti.h) * p.L + grow;
-    const float rho = (p.use_rho && grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
     float m = 0.f, l = 0.f;
-    for (int j = 0; j < ti.n; ++j, ++g) {
+    for (int j = 0; !ti.bad && j < ti.n; ++j, ++g) {
       const int bf = g & 1;
       ok = __all_sync(0xffffffffu, sp_wait(&ctl.s_full[bf], (g >> 1) & 1, ctl, p));
       if (!ok) break;
@@ -363,47 +389,99 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       mbar_arrive(&ctl.p_full[bf]);
     }
     if (!ok) break;
-    // ------------------------------------------------------------- epilogue
-    // The waits that do not need O (the residual tile, the staging slot) are
-    // taken while the tile's last PV runs.
-    const bool r_smem = !p.r_f32 && p.use_r;
+    // hand the tile to the epilogue: slot e holds its counts and (TMEM) its row sums
+    const int e = it & 1;
+    if (it >= 2) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.epi_empty[e], ((it >> 1) - 1) & 1, ctl, p));
+      if (!ok) break;
+    }
+    if (!ti.bad && ti.n > 0) {
+      tmem_st_x1(tL + e, __float_as_uint(l));
+      tmem_wait_st();
+    }
+    if (t == 0) {
+      ctl.epi_n[e] = ti.bad ? 0 : ti.n;
+      ctl.epi_bad[e] = ti.bad;
+    }
+    tc_fence_before();
+    mbar_arrive(&ctl.epi_full[e]);
+  }
+}
+
+// ------------------------------------------------------------------ epilogue
+template <int DPAD>
+__device__ __forceinline__ void sp_epilogue(const TmaSet& tm, const AttnParams& p, SpCtrl& ctl, uint8_t* base,
+                                            uint32_t tmem, int ntiles) {
+  using C = SpCfg<DPAD>;
+  const int t = threadIdx.x - kSpEpiThread0;          // tile row
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tO = tmem + lane_base + C::T_O;
+  const uint32_t tL = tmem + lane_base + C::T_L;
+  uint8_t* sR = base + C::OFF_R;
+  uint8_t* sOst = base + C::OFF_OST;
+  const bool r_smem = !p.r_f32 && p.use_r;
+  uint32_t oi = 0, ri = 0, si = 0;
+  bool ok = true;
+  int it = 0;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+    const int e = it & 1;
+    ok = __all_sync(0xffffffffu, sp_wait(&ctl.epi_full[e], (it >> 1) & 1, ctl, p));
+    if (!ok) break;
+    tc_fence_after();
+    const int n = ctl.epi_n[e];
+    const int bad = ctl.epi_bad[e];
+    float l = 0.f;
+    if (n > 0) {
+      l = __uint_as_float(tmem_ld_x1(tL + e));
+      tmem_wait_ld();
+    }
+    tc_fence_before();
+    mbar_arrive(&ctl.epi_empty[e]);
+    if (bad) continue;
+    int b, h, qb;
+    sp_decode(p, tile, b, h, qb);
+    const int grow = qb * 128 + t;
+    const size_t rho_idx = (static_cast<size_t>(b) * p.H + h) * p.L + grow;
+    const float rho = (p.use_rho && grow < p.L) ? __ldg(p.rho_in + rho_idx) : 0.f;
+    // drain O at once: the next tile's first PV waits for it
+    uint32_t acc[DPAD];
+    if (n > 0) {
+      ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_full, oi & 1, ctl, p));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c + 32 <= DPAD; c += 32) tmem_ld_x32(tO + c, *reinterpret_cast<uint32_t(*)[32]>(&acc[c]));
+      if constexpr (DPAD % 32 != 0)
+        tmem_ld_x16(tO + (DPAD & ~31), *reinterpret_cast<uint32_t(*)[16]>(&acc[DPAD & ~31]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&ctl.o_free);
+      ++oi;
+    }
     if (r_smem) {
       ok = __all_sync(0xffffffffu, sp_wait(&ctl.r_full, ri & 1, ctl, p));
       if (!ok) break;
     }
     // staging slot: thread 0 makes sure the store that last used it has read it
-    const int ss = C::OSTG == 2 ? (si & 1) : 0;
     if (t == 0) {
-      if (C::OSTG == 2) tma_store_wait_read<1>(); else tma_store_wait_read<0>();
+      tma_store_wait_read<0>();
       mbar_arrive(&ctl.stg_ready);
     }
-    if (ti.n > 0) {
-      ok = __all_sync(0xffffffffu, sp_wait(&ctl.o_full, oi & 1, ctl, p));
-      if (!ok) break;
-      tc_fence_after();
-      ++oi;
-    }
     const float rho_hat = p.use_rho ? fminf(1.f, fmaf(rho, p.ramp_mul, p.ramp_add)) : 1.f;
-    const float scale = ti.n > 0 ? rho_hat / l : 0.f;
+    const float scale = n > 0 ? rho_hat / l : 0.f;
     ok = __all_sync(0xffffffffu, sp_wait(&ctl.stg_ready, si & 1, ctl, p));
     if (!ok) break;
-    uint8_t* ost = sOst + ss * C::TILE_BYTES;
-    // 16 columns at a time: O from TMEM, the residual, the bf16 result into the
-    // staging tile (reading more of O per wait measured slower: it spills)
+    uint8_t* ost = sOst;
 #pragma unroll
     for (int c = 0; c < DPAD; c += 16) {
-      uint32_t acc[16];
-      if (ti.n > 0) {
-        tmem_ld_x16(tO + c, acc);
-        tmem_wait_ld();
-      }
       float rr[16];
       if (r_smem) {
         load_row16<DPAD>(sR, 128, t, c, false, rr);
       } else if (p.use_r && grow < p.L) {
         // fp32 residual straight from global memory
         const float4* src = reinterpret_cast<const float4*>(
-            static_cast<const float*>(p.r_in) + ti.b * p.stride_b + ti.h * p.stride_h +
+            static_cast<const float*>(p.r_in) + b * p.stride_b + h * p.stride_h +
             static_cast<long long>(grow) * p.stride_l + c);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -417,8 +495,8 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
       uint32_t pk[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float a0 = (ti.n > 0 ? __uint_as_float(acc[2 * i]) * scale : 0.f) + rr[2 * i];
-        const float a1 = (ti.n > 0 ? __uint_as_float(acc[2 * i + 1]) * scale : 0.f) + rr[2 * i + 1];
+        const float a0 = (n > 0 ? __uint_as_float(acc[c + 2 * i]) * scale : 0.f) + rr[2 * i];
+        const float a1 = (n > 0 ? __uint_as_float(acc[c + 2 * i + 1]) * scale : 0.f) + rr[2 * i + 1];
         pk[i] = pack_bf16x2(a0, a1);
       }
       const bool c1 = c >= 64;
@@ -438,9 +516,9 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
     mbar_arrive(&ctl.stg_full);
     if (t == 0) {
       if (sp_wait(&ctl.stg_full, si & 1, ctl, p)) {
-        const int q_row = ti.qb * 128;
-        tma_store_4d(&tm.o[0], ost, 0, q_row, ti.h, ti.b);
-        if (C::C1) tma_store_4d(&tm.o[1], ost + 128 * 128, 64, q_row, ti.h, ti.b);
+        const int q_row = qb * 128;
+        tma_store_4d(&tm.o[0], ost, 0, q_row, h, b);
+        if (C::C1) tma_store_4d(&tm.o[1], ost + 128 * 128, 64, q_row, h, b);
         tma_store_commit();
       }
     }
@@ -451,7 +529,7 @@ __device__ __forceinline__ void sp_softmax(const TmaSet& tm, const AttnParams& p
 }
 
 template <int DPAD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kSpThreads, 1)
 sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles) {
   using C = SpCfg<DPAD>;
   extern __shared__ uint8_t smem_raw[];
@@ -469,6 +547,8 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
       mbar_init(&ctl.pv_done[i], 1);
       mbar_init(&ctl.ti_full[i], 1);
       mbar_init(&ctl.ti_empty[i], kSoftmaxThreads + 2);
+      mbar_init(&ctl.epi_full[i], kSoftmaxThreads);
+      mbar_init(&ctl.epi_empty[i], kSoftmaxThreads);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&ctl.k_full[i], 1);
@@ -477,6 +557,7 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
       mbar_init(&ctl.v_empty[i], 1);
     }
     mbar_init(&ctl.o_full, 1);
+    mbar_init(&ctl.o_free, kSoftmaxThreads);
     mbar_init(&ctl.r_full, 1);
     mbar_init(&ctl.r_empty, kSoftmaxThreads);
     mbar_init(&ctl.stg_ready, 1);
@@ -485,7 +566,7 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
     ctl.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kSpMmaWarp) {
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -494,16 +575,23 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
 
-  if (warp == kProducerWarp) {
-    sp_producer<DPAD>(tm, p, ctl, base, ntiles);
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) sp_mma<DPAD>(p, ctl, base, tmem, ntiles);
+  if (warp < 4) {
+    reg_alloc<kSpRegsSoftmax>();
+    sp_softmax<DPAD>(p, ctl, tmem, ntiles);
+  } else if (warp < 8) {
+    reg_alloc<kSpRegsEpilogue>();
+    sp_epilogue<DPAD>(tm, p, ctl, base, tmem, ntiles);
   } else {
-    sp_softmax<DPAD>(tm, p, ctl, base, tmem, ntiles);
+    reg_dealloc<kSpRegsOther>();
+    if (warp == kSpProducerWarp) {
+      sp_producer<DPAD>(tm, p, ctl, base, ntiles);
+    } else if (warp == kSpMmaWarp) {
+      if (lane == 0) sp_mma<DPAD>(p, ctl, base, tmem, ntiles);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kSpMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
