@@ -96,10 +96,14 @@ __device__ __forceinline__ void cal_producer(const TmaSet& tm, const AttnParams&
   if (lane > 1) return;
   int issued = 0;
   bool ok = true;
+  // every CTA of a head streams the head's whole K and V: keep them in L2 ahead
+  // of this CTA's own Q (read once)
+  const uint64_t keep = l2_evict_last();
   if (lane == 0) {
+    const uint64_t once = l2_evict_first();
     mbar_arrive_expect_tx(&ctl.q_full, C::TILE);
-    tma_load_4d(base + C::OFF_Q, &tm.q[0], &ctl.q_full, 0, qb * 128, h, b);
-    if (C::C1) tma_load_4d(base + C::OFF_Q + 128 * 128, &tm.q[1], &ctl.q_full, 64, qb * 128, h, b);
+    tma_load_4d_hint(base + C::OFF_Q, &tm.q[0], &ctl.q_full, 0, qb * 128, h, b, once);
+    if (C::C1) tma_load_4d_hint(base + C::OFF_Q + 128 * 128, &tm.q[1], &ctl.q_full, 64, qb * 128, h, b, once);
   }
   CalOrder order{0, ctl.n_kept == p.nkb ? 1 : 0};
   for (int j = 0; j < p.nkb; ++j) {
@@ -111,8 +115,8 @@ __device__ __forceinline__ void cal_producer(const TmaSet& tm, const AttnParams&
     uint8_t* dst = base + C::OFF_STAGE + st * 2 * C::TILE + lane * C::TILE;
     const CUtensorMap* m = lane == 0 ? tm.k : tm.v;
     mbar_arrive_expect_tx(full, C::TILE);
-    tma_load_4d(dst, &m[0], full, 0, kb * 128, h, b);
-    if (C::C1) tma_load_4d(dst + 128 * 128, &m[1], full, 64, kb * 128, h, b);
+    tma_load_4d_hint(dst, &m[0], full, 0, kb * 128, h, b, keep);
+    if (C::C1) tma_load_4d_hint(dst + 128 * 128, &m[1], full, 64, kb * 128, h, b, keep);
     issued = j + 1;
   }
   if (!ok) {
@@ -384,13 +388,15 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
   if (t == 0) {
     if (sp_wait(&ctl.epi, 0, ctl, p) && !ctl.abort_flag) {
       const int q_row = qb * 128;
-      tma_store_4d(&tm.o[0], sO, 0, q_row, h, b);
-      if (C::C1) tma_store_4d(&tm.o[1], sO + 128 * 128, 64, q_row, h, b);
+      const uint64_t once = l2_evict_first();       // outputs: written once, not re-read here
+      tma_store_4d_hint(&tm.o[0], sO, 0, q_row, h, b, once);
+      if (C::C1) tma_store_4d_hint(&tm.o[1], sO + 128 * 128, 64, q_row, h, b, once);
       if (p.r_f32) {
-        for (int c = 0; c < (DPAD + 31) / 32; ++c) tma_store_4d(&tm.r[c], sRst + c * 128 * 128, c * 32, q_row, h, b);
+        for (int c = 0; c < (DPAD + 31) / 32; ++c)
+          tma_store_4d_hint(&tm.r[c], sRst + c * 128 * 128, c * 32, q_row, h, b, once);
       } else {
-        tma_store_4d(&tm.r[0], sRst, 0, q_row, h, b);
-        if (C::C1) tma_store_4d(&tm.r[1], sRst + 128 * 128, 64, q_row, h, b);
+        tma_store_4d_hint(&tm.r[0], sRst, 0, q_row, h, b, once);
+        if (C::C1) tma_store_4d_hint(&tm.r[1], sRst + 128 * 128, 64, q_row, h, b, once);
       }
       tma_store_commit();
       tma_store_wait0();
