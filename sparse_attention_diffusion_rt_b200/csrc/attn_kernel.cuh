@@ -44,6 +44,11 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kMaxKeyBlocks = 4096;
 constexpr float kRescaleLog2 = 8.0f;
+// Every p of a row block is at most the block's row sum (p >= 0, and a rounded
+// sum of non-negative terms is no smaller than any of them), and x > 8 gives
+// p = 2^x > 255.  A block whose row sums are all <= 255 therefore needs no
+// rescale, and only then is its largest x taken (exactly) at all.
+constexpr float kRescaleSum = 255.0f;
 constexpr uint32_t kTmemCols = 512;
 
 struct TmaSet {

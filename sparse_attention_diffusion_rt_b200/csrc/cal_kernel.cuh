@@ -254,10 +254,10 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     if (j == tail_j) mask_tail<128>(s, tail_valid);
     if (j == 0) m = row_max<128>(s) * sl2;
     // P(j) over the first 64 logit columns (the logits are in registers), with
-    // the running max; xmax, the block's largest x = s * sl2 - m, tells whether
-    // that max was too small
-    float xmax;
-    float sum = exp_pack_store_mx<128>(s, sl2, m, tS, xmax);
+    // the running max.  If the row sum exceeds kRescaleSum, the block's largest
+    // x = s * sl2 - m tells whether that max was too small.
+    float sum = exp_pack_store<128>(s, sl2, m, tS);
+    const float xmax = __any_sync(0xffffffffu, sum > kRescaleSum) ? xmax_of<128>(s, sl2, m) : 0.f;
     if (__any_sync(0xffffffffu, xmax > kRescaleLog2)) {
       // rare: the block raised the max by more than 2^8: rescale, then redo P(j)
       tmem_wait_st();                         // the first P(j) stores land before they are redone

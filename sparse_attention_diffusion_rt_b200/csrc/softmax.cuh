@@ -105,6 +105,16 @@ __device__ __forceinline__ float exp_pack_store_mx(const uint32_t (&s)[BN], floa
   return lo + hi;
 }
 
+// Largest x = s_c * sl2 - m of the row block.  x is one rounded fma, monotone
+// in s_c for sl2 > 0, so this is exactly the largest x the exponentials used.
+// (Taken from the raw logits, not from the x values, so that the compiler does
+// not keep the block's 128 x values live from the exponentials to this rare
+// check.)
+template <int BN>
+__device__ __forceinline__ float xmax_of(const uint32_t (&s)[BN], float sl2, float m) {
+  return fmaf(row_max<BN>(s), sl2, -m);
+}
+
 // Load BN fp32 logits of this thread's row from TMEM (caller waits with tmem_wait_ld).
 template <int BN>
 __device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[BN]) {
