@@ -79,21 +79,30 @@ struct SpCfg {
 // Roles of the sparse-step kernel: three warpgroups.  Each sub-partition of
 // the SM holds one warp of each, so the launch gives every thread 168
 // registers (3 x 32 x 168 of a sub-partition's 16384); the warpgroups then
-// rebalance: the softmax holds a 128-logit row in registers and takes 240, the
-// epilogue a whole O row and takes 176, the producer / MMA warpgroup gives
-// back down to 88.  128 x (240 + 176 + 88) = 64512 = 384 x 168: the .inc of
-// the first two exactly use what the .dec of the third returns.
+// rebalance: the softmax holds a 128-logit row in registers, the epilogue a
+// whole O row, the producer / MMA warpgroup gives back down to 80.  The split
+// between the first two follows the head dimension (the epilogue's row is DPAD
+// wide): 248 / 176 at DPAD 128, 256 / 168 below; either way 128 x (softmax +
+// epilogue + 80) = 64512 = 384 x 168, the .inc of the first two exactly using
+// what the .dec of the third returns.
 constexpr int kSpThreads = 384;
 constexpr int kSpEpiThread0 = 128;     // warps 4-7: epilogue
 constexpr int kSpProducerWarp = 8;
 constexpr int kSpMmaWarp = 9;          // warps 10-11 idle
-constexpr uint32_t kSpRegsLaunch = 168, kSpRegsSoftmax = 240, kSpRegsEpilogue = 176, kSpRegsOther = 88;
-static_assert(kSpRegsLaunch * kSpThreads <= 65536 && 3 * 32 * kSpRegsLaunch <= 16384,
-              "launch registers fit the register file and each sub-partition");
-static_assert(32 * (kSpRegsSoftmax + kSpRegsEpilogue + kSpRegsOther) <= 16384,
-              "after the split, one warp of each warpgroup still fits a sub-partition");
-static_assert(128 * (kSpRegsSoftmax + kSpRegsEpilogue + kSpRegsOther) <= kSpThreads * kSpRegsLaunch,
-              "the warpgroups' shares fit the pool the CTA was launched with");
+constexpr uint32_t kSpRegsLaunch = 168, kSpRegsOther = 80;
+template <int DPAD>
+struct SpRegs {
+  static constexpr uint32_t softmax = DPAD == 128 ? 248 : 256;
+  static constexpr uint32_t epilogue = DPAD == 128 ? 176 : 168;
+  static_assert(kSpRegsLaunch * kSpThreads <= 65536 && 3 * 32 * kSpRegsLaunch <= 16384,
+                "launch registers fit the register file and each sub-partition");
+  static_assert(32 * (softmax + epilogue + kSpRegsOther) <= 16384,
+                "after the split, one warp of each warpgroup still fits a sub-partition");
+  static_assert(128 * (softmax + epilogue + kSpRegsOther) <= kSpThreads * kSpRegsLaunch,
+                "the warpgroups' shares fit the pool the CTA was launched with");
+  static_assert(softmax % 8 == 0 && epilogue % 8 == 0 && kSpRegsOther % 8 == 0 && softmax <= 256,
+                "setmaxnreg counts");
+};
 
 struct SpTile {
   int b, h, qb, n, start, bad;
@@ -365,10 +374,10 @@ __device__ __forceinline__ void sp_softmax(const AttnParams& p, SpCtrl& ctl, uin
       mask_tail<128>(s, (j == ti.tail_j) ? ti.tail_valid : 128);
       if (j == 0) m = row_max<128>(s) * sl2;
       // P(g) over the first 64 columns of its own logits (they are in registers),
-      // with the running max; xmax, the block's largest s * sl2 - m, tells
-      // whether that max was too small
-      float xmax;
-      float sum = exp_pack_store_mx<128>(s, sl2, m, tS + 128u * bf, xmax);
+      // with the running max.  If the row sum exceeds kRescaleSum, the block's
+      // largest x = s * sl2 - m tells whether that max was too small.
+      float sum = exp_pack_store<128>(s, sl2, m, tS + 128u * bf);
+      const float xmax = __any_sync(0xffffffffu, sum > kRescaleSum) ? xmax_of<128>(s, sl2, m) : 0.f;
       if (__any_sync(0xffffffffu, xmax > kRescaleLog2)) {
         // rare: the block raised the max by more than 2^8: rescale O, then redo P(g)
         tmem_wait_st();                       // the first P(g) stores land before they are redone
@@ -576,10 +585,10 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
   const uint32_t tmem = ctl.tmem_base;
 
   if (warp < 4) {
-    reg_alloc<kSpRegsSoftmax>();
+    reg_alloc<SpRegs<DPAD>::softmax>();
     sp_softmax<DPAD>(p, ctl, tmem, ntiles);
   } else if (warp < 8) {
-    reg_alloc<kSpRegsEpilogue>();
+    reg_alloc<SpRegs<DPAD>::epilogue>();
     sp_epilogue<DPAD>(tm, p, ctl, base, tmem, ntiles);
   } else {
     reg_dealloc<kSpRegsOther>();
