@@ -202,6 +202,16 @@ template <uint32_t N>
 __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// A warpgroup launched with FROM registers per thread moves to TO: .inc may
+// only raise the count and .dec only lower it (the wrong one is an illegal
+// instruction that no compiler check catches), so the direction follows from
+// the two counts, and equal counts need nothing.
+template <uint32_t FROM, uint32_t TO>
+__device__ __forceinline__ void reg_set() {
+  static_assert(TO % 8 == 0 && TO >= 24 && TO <= 256, "setmaxnreg count");
+  if constexpr (TO > FROM) reg_alloc<TO>();
+  else if constexpr (TO < FROM) reg_dealloc<TO>();
+}
 
 __device__ __forceinline__ uint32_t tmem_ld_x1(uint32_t taddr) {
   uint32_t r;

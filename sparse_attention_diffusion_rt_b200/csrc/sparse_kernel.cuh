@@ -585,13 +585,13 @@ sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntiles)
   const uint32_t tmem = ctl.tmem_base;
 
   if (warp < 4) {
-    reg_alloc<SpRegs<DPAD>::softmax>();
+    reg_set<kSpRegsLaunch, SpRegs<DPAD>::softmax>();
     sp_softmax<DPAD>(p, ctl, tmem, ntiles);
   } else if (warp < 8) {
-    reg_alloc<SpRegs<DPAD>::epilogue>();
+    reg_set<kSpRegsLaunch, SpRegs<DPAD>::epilogue>();
     sp_epilogue<DPAD>(tm, p, ctl, base, tmem, ntiles);
   } else {
-    reg_dealloc<kSpRegsOther>();
+    reg_set<kSpRegsLaunch, kSpRegsOther>();
     if (warp == kSpProducerWarp) {
       sp_producer<DPAD>(tm, p, ctl, base, ntiles);
     } else if (warp == kSpMmaWarp) {
