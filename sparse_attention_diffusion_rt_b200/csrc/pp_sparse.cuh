@@ -8,9 +8,9 @@
 // barrier latency and tensor-core work.  CTA c handles tiles c + i*gridDim.x;
 // even i go to pipeline A, odd i to B.
 //
-// Threads (352): warps 0-3 softmax + epilogue of A, warps 4-7 of B (thread t
+// Threads (384): warps 0-3 softmax + epilogue of A, warps 4-7 of B (thread t
 // owns TMEM lane t % 128), lanes 0 and 1 of warp 8 are the TMA producers of A
-// and B, lane 0 of warps 9 and 10 issue the MMAs of A and B.
+// and B, lane 0 of warps 9 and 10 issue the MMAs of A and B, warp 11 idles.
 // TMEM: pipeline p uses columns [256p, 256p+256): S logits [0,128), bf16 P
 // [128,192), O [192,256).  A pipeline's next QK^T is issued as soon as its
 // softmax has read the current logits (s_free), so it runs under that softmax;
@@ -30,9 +30,19 @@
 
 namespace rtb {
 
-constexpr int kPpThreads = 352;
+constexpr int kPpThreads = 384;
 constexpr int kPpProducerWarp = 8;
-constexpr int kPpMmaWarp = 9;        // warps 9 and 10: MMA issuers of pipelines A and B
+constexpr int kPpMmaWarp = 9;        // warps 9 and 10: MMA issuers of pipelines A and B; warp 11 idle
+// Registers: three warps per sub-partition cap the launch at 168 per thread;
+// the two softmax warpgroups take 216 and the producer / MMA warpgroup gives
+// back down to 56: 128 x (2 x 216 + 56) = 62464 <= 384 x 168.
+constexpr uint32_t kPpRegsLaunch = 168, kPpRegsSoftmax = 216, kPpRegsOther = 56;
+static_assert(kPpRegsLaunch * kPpThreads <= 65536 && 3 * 32 * kPpRegsLaunch <= 16384,
+              "launch registers fit the register file and each sub-partition");
+static_assert(32 * (2 * kPpRegsSoftmax + kPpRegsOther) <= 16384,
+              "after the split, two softmax warps and one other warp still fit a sub-partition");
+static_assert(128 * (2 * kPpRegsSoftmax + kPpRegsOther) <= kPpThreads * kPpRegsLaunch,
+              "the warpgroups' shares fit the pool the CTA was launched with");
 
 struct PpCfg {
   static constexpr int TILE = 128 * 64 * 2;                 // bf16 [128][64]
@@ -407,13 +417,17 @@ pp_sparse_kernel(const __grid_constant__ TmaSet tm, const AttnParams p, int ntil
   const uint32_t tmem = ctl.tmem_base;
 
   if (warp < 8) {
+    reg_set<kPpRegsLaunch, kPpRegsSoftmax>();
     const int pipe = warp >> 2;
     pp_softmax(tm, p, ctl, pipes + pipe * C::PIPE_BYTES, tmem, pipe, ntiles);
-  } else if (warp == kPpProducerWarp) {
-    if (lane < 2) pp_producer(tm, p, ctl, pipes + lane * C::PIPE_BYTES, lane, ntiles);
-  } else if (lane == 0) {
-    const int pipe = warp - kPpMmaWarp;
-    pp_mma(p, ctl, pipes + pipe * C::PIPE_BYTES, tmem, pipe, ntiles);
+  } else {
+    reg_set<kPpRegsLaunch, kPpRegsOther>();
+    if (warp == kPpProducerWarp) {
+      if (lane < 2) pp_producer(tm, p, ctl, pipes + lane * C::PIPE_BYTES, lane, ntiles);
+    } else if (warp < kPpMmaWarp + 2 && lane == 0) {
+      const int pipe = warp - kPpMmaWarp;
+      pp_mma(p, ctl, pipes + pipe * C::PIPE_BYTES, tmem, pipe, ntiles);
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -65,46 +65,6 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BN], float s
   return lo + hi;
 }
 
-// As exp_pack_store, and also returns in xmax the largest x = s_c * sl2 - m of
-// the row block, so that a running max that is too small (x above the lazy
-// rescale threshold) is detected without a separate max pass: the max is taken
-// on the ALU pipe while the MUFU computes the exponentials.
-template <int BN>
-__device__ __forceinline__ float exp_pack_store_mx(const uint32_t (&s)[BN], float sl2, float m, uint32_t tP,
-                                                   float& xmax) {
-  uint64_t sum[4];
-  float mx[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    sum[i] = 0ull;
-    mx[i] = -INFINITY;
-  }
-  const uint64_t scale2 = f2_pack(sl2, sl2);
-  const uint64_t neg_m2 = f2_pack(-m, -m);
-#pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 64) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const uint64_t x = ffma2(f2_pack(__uint_as_float(s[c0 + 2 * c]), __uint_as_float(s[c0 + 2 * c + 1])),
-                               scale2, neg_m2);
-      float x0, x1;
-      f2_unpack(x, x0, x1);
-      mx[c & 3] = max3f(mx[c & 3], x0, x1);
-      const float p0 = ex2_approx(x0);
-      const float p1 = ex2_approx(x1);
-      sum[c & 3] = fadd2(sum[c & 3], f2_pack(p0, p1));
-      pk[c] = pack_bf16x2(p0, p1);
-    }
-    tmem_st_x32(tP + c0 / 2, pk);
-  }
-  xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-  const uint64_t t = fadd2(fadd2(sum[0], sum[1]), fadd2(sum[2], sum[3]));
-  float lo, hi;
-  f2_unpack(t, lo, hi);
-  return lo + hi;
-}
-
 // Largest x = s_c * sl2 - m of the row block.  x is one rounded fma, monotone
 // in s_c for sl2 > 0, so this is exactly the largest x the exponentials used.
 // (Taken from the raw logits, not from the x values, so that the compiler does
@@ -141,11 +101,10 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float alpha) {
 
 namespace rtb {
 
-// Two-pass variants that keep at most 64 logits in registers: the row max is
-// taken over S read from TMEM in two halves, then S is read again, half by half,
-// exponentiated and written back as bf16 P into the first BN/2 columns of the
-// same TMEM region (column 16c of P overwrites logits that were already read),
-// so that P needs no TMEM of its own.  Keys c >= valid are excluded.
+// Two-pass form for a softmax that keeps at most 64 logits in registers: the row
+// max is taken over S read from TMEM in two halves (row_max_tmem), then S is
+// read again, half by half, and exponentiated (exp_pass_tmem_sep).  Keys
+// c >= valid are excluded.
 template <int BN>
 __device__ __forceinline__ float row_max_tmem(uint32_t tS, int valid) {
   float mx[8];
@@ -171,10 +130,11 @@ __device__ __forceinline__ float row_max_tmem(uint32_t tS, int valid) {
   return max3f(a, b, fmaxf(mx[6], mx[7]));
 }
 
-// As exp_pass_tmem but P goes to its own TMEM columns tP; on_s_read() runs once
-// the last logits have been read (S may then be overwritten by the next QK^T),
-// before_p() runs before the first P store (P's previous contents must have been
-// consumed).
+// p_c = 2^(s_c * sl2 - m) for a row block whose logits are read from TMEM (tS)
+// in halves of 64, keys c >= valid excluded; P goes as bf16 pairs to its own
+// TMEM columns tP.  on_s_read() runs once the last logits have been read (S may
+// then be overwritten by the next QK^T), before_p() before the first P store
+// (P's previous contents must have been consumed).  Returns sum_c p_c.
 template <int BN, typename OnSRead, typename BeforeP>
 __device__ __forceinline__ float exp_pass_tmem_sep(uint32_t tS, uint32_t tP, float sl2, float m, int valid,
                                                    OnSRead on_s_read, BeforeP before_p) {
@@ -208,43 +168,6 @@ __device__ __forceinline__ float exp_pass_tmem_sep(uint32_t tS, uint32_t tP, flo
     }
     if (h0 == 0) before_p();
     tmem_st_x32(tP + h0 / 2, pk);
-  }
-  const uint64_t t = fadd2(fadd2(sum[0], sum[1]), fadd2(sum[2], sum[3]));
-  float lo, hi;
-  f2_unpack(t, lo, hi);
-  return lo + hi;
-}
-
-template <int BN>
-__device__ __forceinline__ float exp_pass_tmem(uint32_t tS, float sl2, float m, int valid) {
-  uint64_t sum[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) sum[i] = 0ull;
-  const uint64_t scale2 = f2_pack(sl2, sl2);
-  const uint64_t neg_m2 = f2_pack(-m, -m);
-#pragma unroll
-  for (int h0 = 0; h0 < BN; h0 += 64) {
-    uint32_t s[64];
-    tmem_ld_x32(tS + h0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-    tmem_ld_x32(tS + h0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-    tmem_wait_ld();
-    if (valid < h0 + 64) {
-#pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (h0 + c >= valid) s[c] = __float_as_uint(-INFINITY);
-    }
-    uint32_t pk[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const uint64_t x = ffma2(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), scale2, neg_m2);
-      float x0, x1;
-      f2_unpack(x, x0, x1);
-      const float p0 = ex2_approx(x0);
-      const float p1 = ex2_approx(x1);
-      sum[c & 3] = fadd2(sum[c & 3], f2_pack(p0, p1));
-      pk[c] = pack_bf16x2(p0, p1);
-    }
-    tmem_st_x32(tS + h0 / 2, pk);      // P columns [h0/2, h0/2 + 32): logits already consumed
   }
   const uint64_t t = fadd2(fadd2(sum[0], sum[1]), fadd2(sum[2], sum[3]));
   float lo, hi;
