@@ -78,8 +78,12 @@ __device__ __forceinline__ float xmax_of(const uint32_t (&s)[BN], float sl2, flo
 // Load BN fp32 logits of this thread's row from TMEM (caller waits with tmem_wait_ld).
 template <int BN>
 __device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[BN]) {
+  if constexpr (BN == 128) {
+    tmem_ld_x128(tS, s);
+  } else {
 #pragma unroll
-  for (int c = 0; c < BN; c += 32) tmem_ld_x32(tS + c, *reinterpret_cast<uint32_t(*)[32]>(&s[c]));
+    for (int c = 0; c < BN; c += 32) tmem_ld_x32(tS + c, *reinterpret_cast<uint32_t(*)[32]>(&s[c]));
+  }
 }
 
 // Rescale one TMEM accumulator row (this thread's lane) by alpha.
