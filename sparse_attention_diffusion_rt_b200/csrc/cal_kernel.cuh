@@ -257,8 +257,10 @@ __device__ __forceinline__ void cal_softmax(const TmaSet& tm, const AttnParams& 
     // the running max.  If the row sum exceeds kRescaleSum, the block's largest
     // x = s * sl2 - m tells whether that max was too small.
     float sum = exp_pack_store<128>(s, sl2, m, tS);
-    const float xmax = __any_sync(0xffffffffu, sum > kRescaleSum) ? xmax_of<128>(s, sl2, m) : 0.f;
-    if (__any_sync(0xffffffffu, xmax > kRescaleLog2)) {
+    // chk is the same in every lane, so all lanes or none take the second vote
+    const bool chk = __any_sync(0xffffffffu, sum > kRescaleSum);
+    const float xmax = chk ? xmax_of<128>(s, sl2, m) : 0.f;
+    if (chk && __any_sync(0xffffffffu, xmax > kRescaleLog2)) {
       // rare: the block raised the max by more than 2^8: rescale, then redo P(j)
       tmem_wait_st();                         // the first P(j) stores land before they are redone
       const float m_new = m + fmaxf(xmax, 0.f);
